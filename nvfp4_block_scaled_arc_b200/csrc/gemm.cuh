@@ -1,0 +1,328 @@
+// gemm.cuh -- the compute-bound half of the hot path: one persistent, warp-specialised
+// tcgen05 GEMM skeleton instantiated twice.
+//   FP4 = true:  block-scaled NVFP4 GEMM of depth K_aug (tcgen05.mma kind::mxf4nvf4,
+//                scale_vec::4X: one E4M3 scale per 16 elements of A and of B), the unified
+//                GEMM of "ARCQuant ... Augmented Residual Channels" (Unified GEMM Executie:
+//                one GEMM over K_in + S absorbs the residual correction by linearity), epilogue
+//                Y = bf16(s_A s_B acc [+ add]).
+//   FP4 = false: BF16 GEMM (tcgen05.mma kind::f16), the reference-precision switch of RAMP
+//                (section 4.1: the recurrent steps after the switch run in BF16).
+//
+// CTA = 6 warps, one CTA per SM, persistent over 128 x 256 output tiles (grouped raster):
+//   warp 0      TMA producer: A tile 128 rows x 128 bytes and B tile 256 rows x 128 bytes per
+//               stage (128-byte swizzle), plus the stage's scale atoms as 1-D bulk copies (A:
+//               up to 4 atoms of its 128-row block, B: up to 4 atoms of each of its two
+//               128-row blocks); no multicast.
+//   warp 1      TMEM allocation and MMA issue (one thread): per stage, tcgen05.cp of the scale
+//               atoms into TMEM (32x128b, replicated to the four lane quarters), then 4 MMAs of
+//               K = 64 (fp4) / 16 (bf16), committed to the stage's "empty" barrier.
+//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (warp w owns TMEM lanes
+//               32*(w%4)..+31 = tile rows), scale by alpha, optional residual add, bf16 stores.
+// TMEM: fp32 accumulator 128 lanes x 256 columns (two of them for bf16; fp4 keeps one and puts
+// the scale factors in columns 256..303). Every wait is bounded (wait_ns); a wait that runs out
+// raises the CTA's abort flag and the device status word, and the CTA drains what it issued
+// and frees its tensor memory before it returns.
+#pragma once
+
+#include "arc_device.cuh"
+
+namespace arc {
+
+template <bool FP4>
+struct GemmTraits;
+
+template <>
+struct GemmTraits<true> {
+  static constexpr int BM = 128, BN = 256, STAGES = 4, ACC_STAGES = 1;
+  static constexpr int A_BYTES = BM * 128, B_BYTES = BN * 128;
+  static constexpr int SFA_BYTES = 4 * 512, SFB_BYTES = 2 * 4 * 512;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr uint32_t IDESC = idesc_nvf4(BM, BN);
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int SFA_COL = 256, SFB_COL = 272;
+};
+
+template <>
+struct GemmTraits<false> {
+  static constexpr int BM = 128, BN = 256, STAGES = 4, ACC_STAGES = 2;
+  static constexpr int A_BYTES = BM * 128, B_BYTES = BN * 128;
+  static constexpr int SFA_BYTES = 0, SFB_BYTES = 0;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t IDESC = idesc_bf16(BM, BN);
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int SFA_COL = 0, SFB_COL = 0;
+};
+
+template <bool FP4>
+constexpr int gemm_smem_bytes() {
+  return GemmTraits<FP4>::STAGES * GemmTraits<FP4>::STAGE_BYTES + 1024 + 256;
+}
+
+struct GemmArgs {
+  int M, N;
+  int ksteps;   // MMA K-steps over the whole depth
+  int kstages;  // pipeline stages per tile (4 K-steps each)
+  int katoms;   // fp4: 512-byte scale atoms per 128-row block (K_pad / 64)
+  int nblk128;  // fp4: 128-row blocks of B's scales (ceil(N / 128))
+  int tiles_m, tiles_n;
+  int box_rows_a, box_rows_b;  // TMA box heights (min(128, M), min(256, N))
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  const float* a_scale;
+  const float* b_scale;
+  __nv_bfloat16* y;
+  int64_t ldy;
+  const __nv_bfloat16* add;
+  int64_t ld_add;
+  uint64_t wait_ns;
+  int inject;
+};
+
+__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int& tm, int& tn) {
+  constexpr int GM = 16;  // consecutive tiles walk 16 row blocks before moving to the next column block
+  const int per_group = GM * tiles_n;
+  const int group = t / per_group;
+  const int first_m = group * GM;
+  const int gm = min(GM, tiles_m - first_m);
+  const int rr = t - group * per_group;
+  tm = first_m + rr % gm;
+  tn = rr / gm;
+}
+
+// Wait used only while tearing down after an abort: bounded by time, ignores the abort flag.
+__device__ __forceinline__ void mbar_wait_teardown(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_test(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) return;
+  }
+}
+
+template <bool FP4, bool ADD>
+__global__ void __launch_bounds__(192, 1)
+    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
+  using T = GemmTraits<FP4>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + T::STAGES * T::STAGE_BYTES);
+  uint64_t* empty = full + T::STAGES;
+  uint64_t* acc_full = empty + T::STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < T::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, T::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int ntiles = g.tiles_m * g.tiles_n;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------------ producer
+      uint32_t stage = 0, phase = 0, armed = 0, armed_par = 0;
+      bool skip = (g.inject == 1) && blockIdx.x == 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        int tm, tn;
+        tile_coords(t, g.tiles_m, g.tiles_n, tm, tn);
+        for (int ks = 0; ks < g.kstages; ++ks) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, g.wait_ns, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sA = smem + stage * T::STAGE_BYTES;
+          uint8_t* sB = sA + T::A_BYTES;
+          if (skip) {
+            skip = false;  // failure injection: this stage's loads are never issued
+          } else {
+            uint32_t bytes = static_cast<uint32_t>(g.box_rows_a + g.box_rows_b) * 128u;
+            int natoms = 0, nb = 0;
+            if (FP4) {
+              natoms = min(4, g.katoms - 4 * ks);
+              nb = min(2, g.nblk128 - 2 * tn);
+              bytes += static_cast<uint32_t>(natoms * 512 * (1 + nb));
+            }
+            mbar_arrive_expect_tx(&full[stage], bytes);
+            const int kx = FP4 ? ks * 128 : ks * 64;
+            tma_load_2d(sA, &tmA, &full[stage], kx, tm * T::BM);
+            tma_load_2d(sB, &tmB, &full[stage], kx, tn * T::BN);
+            if (FP4) {
+              uint8_t* sSFA = sB + T::B_BYTES;
+              uint8_t* sSFB = sSFA + T::SFA_BYTES;
+              bulk_load(sSFA, g.sfa + (static_cast<int64_t>(tm) * g.katoms + 4 * ks) * 512, natoms * 512, &full[stage]);
+              for (int b = 0; b < nb; ++b)
+                bulk_load(sSFB + b * 2048, g.sfb + (static_cast<int64_t>(2 * tn + b) * g.katoms + 4 * ks) * 512,
+                          natoms * 512, &full[stage]);
+            }
+            armed |= 1u << stage;
+            armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          }
+          if (++stage == T::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (*abort_flag) {
+        // let every load this thread issued land before the CTA goes away
+        for (int s = 0; s < T::STAGES; ++s)
+          if ((armed >> s) & 1u) mbar_wait_teardown(&full[s], (armed_par >> s) & 1u, g.wait_ns);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------------ MMA issuer
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, g.wait_ns, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + acc * T::BN;
+        for (int ks = 0; ks < g.kstages; ++ks) {
+          if (!mbar_wait(&full[stage], phase, g.wait_ns, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint8_t* sA = smem + stage * T::STAGE_BYTES;
+          uint8_t* sB = sA + T::A_BYTES;
+          const int nk = FP4 ? min(4, g.ksteps - 4 * ks) : 4;
+          if (FP4) {
+            uint8_t* sSFA = sB + T::B_BYTES;
+            uint8_t* sSFB = sSFA + T::SFA_BYTES;
+            for (int k = 0; k < nk; ++k) {
+              tc_cp_sf_atom(tmem + T::SFA_COL + 4 * k, desc_sf_atom(smem_u32(sSFA + k * 512)));
+              tc_cp_sf_atom(tmem + T::SFB_COL + 8 * k, desc_sf_atom(smem_u32(sSFB + k * 512)));
+              tc_cp_sf_atom(tmem + T::SFB_COL + 8 * k + 4, desc_sf_atom(smem_u32(sSFB + 2048 + k * 512)));
+            }
+          }
+          const uint64_t da = desc_kmajor_sw128(smem_u32(sA));
+          const uint64_t db = desc_kmajor_sw128(smem_u32(sB));
+          for (int k = 0; k < nk; ++k) {
+            const uint64_t off = static_cast<uint64_t>((k * 32) >> 4);
+            const uint32_t accum = (ks > 0 || k > 0) ? 1u : 0u;
+            if (FP4)
+              tc_mma_nvf4(d_tmem, da + off, db + off, T::IDESC, tmem + T::SFA_COL + 4 * k, tmem + T::SFB_COL + 8 * k,
+                          accum);
+            else
+              tc_mma_bf16(d_tmem, da + off, db + off, T::IDESC, accum);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == T::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&acc_full[acc]);
+        if (++acc == T::ACC_STAGES) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      // nothing issued may still be running when the tensor memory is released
+      tc_commit(drain);
+      mbar_wait_teardown(drain, 0, g.wait_ns);
+    }
+  } else {
+    // -------------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    const float alpha = FP4 ? __fmul_rn(*g.a_scale, *g.b_scale) : 1.0f;
+    uint32_t acc = 0, acc_phase = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      int tm, tn;
+      tile_coords(t, g.tiles_m, g.tiles_n, tm, tn);
+      const int row = tm * T::BM + q * 32 + lane;
+      const bool row_ok = row < g.M;
+      const int col0 = tn * T::BN;
+      uint32_t addv[ADD ? T::BN / 2 : 1];
+      if (ADD) {
+        // residual tile into registers before the accumulator is ready (keeps TMEM hold short)
+#pragma unroll
+        for (int j = 0; j < T::BN / 8; ++j) {
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (row_ok && col0 + 8 * j < g.N)
+            v = *reinterpret_cast<const uint4*>(g.add + static_cast<int64_t>(row) * g.ld_add + col0 + 8 * j);
+          addv[4 * j + 0] = v.x;
+          addv[4 * j + 1] = v.y;
+          addv[4 * j + 2] = v.z;
+          addv[4 * j + 3] = v.w;
+        }
+      }
+      // every lane waits; the warp goes on only if all of them saw the accumulator (the TMEM
+      // loads below are warp-collective, so the decision must be uniform)
+      const bool ready = mbar_wait(&acc_full[acc], acc_phase, g.wait_ns, abort_flag);
+      if (!__all_sync(0xFFFFFFFFu, ready)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * T::BN;
+      __nv_bfloat16* yrow = g.y + static_cast<int64_t>(row) * g.ldy;
+#pragma unroll
+      for (int c = 0; c < T::BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tbase + c * 32, r);
+        tmem_ld_wait();
+        if (c == T::BN / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        }
+        if (row_ok) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int col = col0 + c * 32 + 8 * j;
+            if (col < g.N) {
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(alpha, __uint_as_float(r[8 * j + e]));
+              if (ADD) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  const uint32_t w = addv[(c * 32 + 8 * j + e) >> 1];
+                  f[e] = __fadd_rn(f[e], (e & 1) ? bf16_hi(w) : bf16_lo(w));
+                }
+              }
+              uint4 o;
+              o.x = pack_bf16x2_rn(f[0], f[1]);
+              o.y = pack_bf16x2_rn(f[2], f[3]);
+              o.z = pack_bf16x2_rn(f[4], f[5]);
+              o.w = pack_bf16x2_rn(f[6], f[7]);
+              *reinterpret_cast<uint4*>(yrow + col) = o;
+            }
+          }
+        }
+      }
+      if (++acc == T::ACC_STAGES) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, T::TMEM_COLS);
+  }
+}
+
+}  // namespace arc

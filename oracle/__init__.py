@@ -336,6 +336,17 @@ def gemm_nvfp4_f64(a_codes, a_sf, s_a, b_codes, b_sf, s_b, rows=None, k_range=No
     return y
 
 
+def gemm_nvfp4_f64_matmul(a_codes, a_sf, s_a, b_codes, b_sf, s_b, rows=None) -> np.ndarray:
+    """Same result as gemm_nvfp4_f64 with a library matmul as the summation step: operands are
+    dequantized exactly (E2M1 * E4M3 products are exact in fp32), then an FP64 matmul."""
+    a_codes = np.ascontiguousarray(a_codes)
+    M = a_codes.shape[0]
+    rows = _rows_arg(rows, M)
+    A = dequant(np.ascontiguousarray(a_codes[rows]), np.ascontiguousarray(np.asarray(a_sf)[rows])).astype(np.float64)
+    B = dequant(b_codes, b_sf).astype(np.float64)
+    return (np.float64(np.float32(s_a)) * np.float64(np.float32(s_b))) * (A @ B.T)
+
+
 def gemm_nvfp4_i64(a_codes, a_sf, b_codes, b_sf, rows=None, k_range=None) -> np.ndarray:
     """Exact integer sums sum_k a'b' (a' = 2 E2M1 * 512 E4M3); Y = sum * 2^-20 * s_A s_W."""
     a_codes = np.ascontiguousarray(a_codes)

@@ -1,0 +1,70 @@
+"""The C-ABI library (no GPU needed): it loads, exports every function include/arc.h declares,
+its size queries follow the documented layout, and host-side argument checks reject bad calls
+before any CUDA work."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import nvfp4_block_scaled_arc_b200 as arc
+import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from nvfp4_block_scaled_arc_b200 import _build
+
+    _build.build()
+    return arc.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "arc.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(arc_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(arc.exported_symbols())
+
+
+def test_size_queries(L):
+    for rows, kaug in [(16, 272), (4096, 4224), (130, 14464), (1, 64), (129, 65)]:
+        kp = (kaug + 63) // 64 * 64
+        assert L.arc_kpad(kaug) == kp == O.kpad(kaug)
+        assert L.arc_nvfp4_codes_bytes(rows, kaug) == rows * kp // 2
+        assert L.arc_nvfp4_sf_bytes(rows, kaug) == O.sf_swizzled_bytes(rows, kp // 16)
+    assert L.arc_quantize_workspace_bytes(4096, 128) >= 4 + 4096 * 128 * 4 + 4096 * 8
+    assert L.arc_status_str(5) == b"ARC_ERR_TIMEOUT"
+
+
+def test_host_checks_reject_before_any_launch(L):
+    P = ctypes.c_void_p
+    fake = P(0x10000)  # never dereferenced: the checks return first
+    ws = P(0x20000)
+    # K % 16 != 0
+    assert L.arc_quantize_act_nvfp4(fake, 4, 40, 40, None, 0, None, 1e-6, None, fake, fake, fake, ws, 1 << 20, None) == 1
+    # r % 16 != 0
+    assert L.arc_quantize_act_nvfp4(fake, 4, 64, 64, fake, 8, None, 1e-6, None, fake, fake, fake, ws, 1 << 20, None) == 1
+    # r > K
+    assert L.arc_quantize_act_nvfp4(fake, 4, 64, 64, fake, 80, None, 1e-6, None, fake, fake, fake, ws, 1 << 20, None) == 1
+    # NULL input
+    assert L.arc_quantize_act_nvfp4(None, 4, 64, 64, None, 0, None, 1e-6, None, fake, fake, fake, ws, 1 << 20, None) == 1
+    # misaligned codes
+    assert L.arc_quantize_act_nvfp4(fake, 4, 64, 64, None, 0, None, 1e-6, None, P(0x10008), fake, fake, ws, 1 << 20, None) == 2
+    # workspace too small
+    assert L.arc_quantize_act_nvfp4(fake, 4, 64, 64, None, 0, None, 1e-6, None, fake, fake, fake, ws, 8, None) == 6
+    # GEMM: N % 8 != 0, ldy < N
+    assert L.arc_gemm_nvfp4(fake, fake, fake, fake, fake, fake, 4, 12, 64, fake, 12, None, 0, None) == 1
+    assert L.arc_gemm_bf16(fake, 64, fake, 64, 4, 16, 64, fake, 8, None, 0, None) == 1
+    assert L.arc_gemm_bf16(P(0x10004), 64, fake, 64, 4, 16, 64, fake, 16, None, 0, None) == 2
+    assert L.arc_set_wait_limit_ns(0) == 1
+    assert L.arc_debug_inject(7) == 1

@@ -268,6 +268,13 @@ def test_gemm_linearity_exact():
     np.testing.assert_allclose(y, yi, rtol=1e-12, atol=1e-300)
 
 
+def test_gemm_matmul_form_equals_scalar_loop():
+    d, idx, sa, sw, ac, asf, bc, bsf = _packed_tiny()
+    y1 = O.gemm_nvfp4_f64(ac, asf, sa, bc, bsf, sw)
+    y2 = O.gemm_nvfp4_f64_matmul(ac, asf, sa, bc, bsf, sw, rows=np.arange(16))
+    np.testing.assert_allclose(y2, y1, rtol=1e-12, atol=1e-300)
+
+
 def test_gemm_bruteforce_tiny():
     d, idx, sa, sw, ac, asf, bc, bsf = _packed_tiny()
     kp = ac.shape[1] * 2
