@@ -61,7 +61,8 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 // Wait until the phase with the given parity has completed. Bounded: after limit_ns of
 // wall time (or once another warp of the CTA has raised *abort) it gives up, raises *abort,
 // records a timeout in the status word and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns, volatile int* abort,
+                                          uint32_t sleep_ns = 0) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
@@ -72,6 +73,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
       set_status(kStatusTimeout);
       return false;
     }
+    // long waits (a whole tile) sleep between polls so they leave the issue slots to the
+    // warps that feed the tensor cores
+    if (sleep_ns) __nanosleep(sleep_ns);
   }
 }
 
@@ -256,6 +260,27 @@ __device__ __forceinline__ float e2m1_value(uint32_t c) {
   return (c & 8u) ? -v : v;
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: two IEEE round-to-nearest operations per
+// instruction, no contraction between them).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
 // Correctly rounded x / d from the correctly rounded reciprocal rcp = RN(1/d) with one
 // remainder correction (P. Markstein, "Computation of elementary functions on the IBM
 // RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990: if y is RN(1/d) and q is within
@@ -265,6 +290,13 @@ __device__ __forceinline__ float div_rn_from_rcp(float x, float d, float rcp) {
   const float q = __fmul_rn(x, rcp);
   const float r = __fmaf_rn(-q, d, x);
   return __fmaf_rn(r, rcp, q);
+}
+
+// The same on a pair: x2 / d with nd2 = (-d, -d) and rcp2 = (RN(1/d), RN(1/d)).
+__device__ __forceinline__ uint64_t div2_rn_from_rcp(uint64_t x2, uint64_t nd2, uint64_t rcp2) {
+  const uint64_t q = f2_mul(x2, rcp2);
+  const uint64_t r = f2_fma(q, nd2, x2);
+  return f2_fma(r, rcp2, q);
 }
 
 }  // namespace arc

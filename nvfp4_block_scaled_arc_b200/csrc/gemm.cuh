@@ -8,7 +8,7 @@
 //   FP4 = false: BF16 GEMM (tcgen05.mma kind::f16), the reference-precision switch of RAMP
 //                (section 4.1: the recurrent steps after the switch run in BF16).
 //
-// CTA = 6 warps, one CTA per SM, persistent over 128 x 256 output tiles (grouped raster):
+// CTA = 10 warps, one CTA per SM, persistent over 128 x 256 output tiles (grouped raster):
 //   warp 0      TMA producer: A tile 128 rows x 128 bytes and B tile 256 rows x 128 bytes per
 //               stage (128-byte swizzle), plus the stage's scale atoms as 1-D bulk copies (A:
 //               up to 4 atoms of its 128-row block, B: up to 4 atoms of each of its two
@@ -16,8 +16,9 @@
 //   warp 1      TMEM allocation and MMA issue (one thread): per stage, tcgen05.cp of the scale
 //               atoms into TMEM (32x128b, replicated to the four lane quarters), then 4 MMAs of
 //               K = 64 (fp4) / 16 (bf16), committed to the stage's "empty" barrier.
-//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (warp w owns TMEM lanes
-//               32*(w%4)..+31 = tile rows), scale by alpha, optional residual add, bf16 stores.
+//   warps 2..9  epilogue: tcgen05.ld of the fp32 accumulator (warp w owns TMEM lanes
+//               32*(w%4)..+31 = tile rows, and one 128-column half), scale by alpha, optional
+//               residual add, bf16 stores.
 // TMEM: fp32 accumulator 128 lanes x 256 columns (two of them for bf16; fp4 keeps one and puts
 // the scale factors in columns 256..303). Every wait is bounded (wait_ns); a wait that runs out
 // raises the CTA's abort flag and the device status word, and the CTA drains what it issued
@@ -97,8 +98,10 @@ __device__ __forceinline__ void mbar_wait_teardown(uint64_t* bar, uint32_t parit
   }
 }
 
+constexpr int kGemmThreads = 320;  // producer warp, MMA warp, 8 epilogue warps
+
 template <bool FP4, bool ADD>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
   using T = GemmTraits<FP4>;
   extern __shared__ uint8_t smem_raw[];
@@ -119,7 +122,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4);
+      mbar_init(&acc_empty[a], 8);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -247,20 +250,27 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // -------------------------------------------------------------------- epilogue
+    // 8 warps: warp w reads TMEM lane quarter w%4 (tile rows 32*(w%4)..+31) and column half
+    // (w-2)/4 (128 columns). Without a residual add the warp pulls its whole 32 x 128 block out
+    // of TMEM in one burst and releases the accumulator before it converts and stores; with an
+    // add, the residual block is prefetched into registers and the accumulator is read and
+    // stored 32 columns at a time.
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     const float alpha = FP4 ? __fmul_rn(*g.a_scale, *g.b_scale) : 1.0f;
+    constexpr int HB = T::BN / 2;  // columns per warp
     uint32_t acc = 0, acc_phase = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
       int tm, tn;
       tile_coords(t, g.tiles_m, g.tiles_n, tm, tn);
       const int row = tm * T::BM + q * 32 + lane;
       const bool row_ok = row < g.M;
-      const int col0 = tn * T::BN;
-      uint32_t addv[ADD ? T::BN / 2 : 1];
+      const int col0 = tn * T::BN + half * HB;
+      __nv_bfloat16* yrow = g.y + static_cast<int64_t>(row) * g.ldy;
+      uint32_t addv[ADD ? HB / 2 : 1];
       if (ADD) {
-        // residual tile into registers before the accumulator is ready (keeps TMEM hold short)
 #pragma unroll
-        for (int j = 0; j < T::BN / 8; ++j) {
+        for (int j = 0; j < HB / 8; ++j) {
           uint4 v = make_uint4(0, 0, 0, 0);
           if (row_ok && col0 + 8 * j < g.N)
             v = *reinterpret_cast<const uint4*>(g.add + static_cast<int64_t>(row) * g.ld_add + col0 + 8 * j);
@@ -272,42 +282,74 @@ __global__ void __launch_bounds__(192, 1)
       }
       // every lane waits; the warp goes on only if all of them saw the accumulator (the TMEM
       // loads below are warp-collective, so the decision must be uniform)
-      const bool ready = mbar_wait(&acc_full[acc], acc_phase, g.wait_ns, abort_flag);
+      const bool ready = mbar_wait(&acc_full[acc], acc_phase, g.wait_ns, abort_flag, 64);
       if (!__all_sync(0xFFFFFFFFu, ready)) break;
       tc_fence_after();
-      const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * T::BN;
-      __nv_bfloat16* yrow = g.y + static_cast<int64_t>(row) * g.ldy;
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * T::BN + half * HB;
+      if (!ADD) {
+        uint32_t r[HB / 32][32];
 #pragma unroll
-      for (int c = 0; c < T::BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tbase + c * 32, r);
+        for (int c = 0; c < HB / 32; ++c) tmem_ld_32x32b_x32(tbase + c * 32, r[c]);
         tmem_ld_wait();
-        if (c == T::BN / 32 - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[acc]);
-        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
         if (row_ok) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int col = col0 + c * 32 + 8 * j;
-            if (col < g.N) {
-              float f[8];
+          for (int c = 0; c < HB / 32; ++c) {
 #pragma unroll
-              for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(alpha, __uint_as_float(r[8 * j + e]));
-              if (ADD) {
+            for (int j = 0; j < 4; ++j) {
+              const int col = col0 + c * 32 + 8 * j;
+              if (col < g.N) {
+                uint64_t f[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  f[e] = f2_mul(f2_pack(__uint_as_float(r[c][8 * j + 2 * e]), __uint_as_float(r[c][8 * j + 2 * e + 1])),
+                                f2_pack(alpha, alpha));
+                uint4 o;
+                float a0, a1;
+                f2_unpack(f[0], a0, a1);
+                o.x = pack_bf16x2_rn(a0, a1);
+                f2_unpack(f[1], a0, a1);
+                o.y = pack_bf16x2_rn(a0, a1);
+                f2_unpack(f[2], a0, a1);
+                o.z = pack_bf16x2_rn(a0, a1);
+                f2_unpack(f[3], a0, a1);
+                o.w = pack_bf16x2_rn(a0, a1);
+                *reinterpret_cast<uint4*>(yrow + col) = o;
+              }
+            }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < HB / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tbase + c * 32, r);
+          tmem_ld_wait();
+          if (c == HB / 32 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+          }
+          if (row_ok) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int col = col0 + c * 32 + 8 * j;
+              if (col < g.N) {
+                float f[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                   const uint32_t w = addv[(c * 32 + 8 * j + e) >> 1];
-                  f[e] = __fadd_rn(f[e], (e & 1) ? bf16_hi(w) : bf16_lo(w));
+                  f[e] = __fadd_rn(__fmul_rn(alpha, __uint_as_float(r[8 * j + e])), (e & 1) ? bf16_hi(w) : bf16_lo(w));
                 }
+                uint4 o;
+                o.x = pack_bf16x2_rn(f[0], f[1]);
+                o.y = pack_bf16x2_rn(f[2], f[3]);
+                o.z = pack_bf16x2_rn(f[4], f[5]);
+                o.w = pack_bf16x2_rn(f[6], f[7]);
+                *reinterpret_cast<uint4*>(yrow + col) = o;
               }
-              uint4 o;
-              o.x = pack_bf16x2_rn(f[0], f[1]);
-              o.y = pack_bf16x2_rn(f[2], f[3]);
-              o.z = pack_bf16x2_rn(f[4], f[5]);
-              o.w = pack_bf16x2_rn(f[6], f[7]);
-              *reinterpret_cast<uint4*>(yrow + col) = o;
             }
           }
         }

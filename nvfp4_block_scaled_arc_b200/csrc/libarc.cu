@@ -52,7 +52,11 @@ arc_status device_check(int* sms) {
         cudaFuncSetAttribute(arc::k_gemm<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              arc::gemm_smem_bytes<false>()) != cudaSuccess ||
         cudaFuncSetAttribute(arc::k_gemm<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             arc::gemm_smem_bytes<false>()) != cudaSuccess)
+                             arc::gemm_smem_bytes<false>()) != cudaSuccess ||
+        cudaFuncSetAttribute(arc::k_quant_stream<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             arc::kQuantSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(arc::k_quant_stream<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             arc::kQuantSmem) != cudaSuccess)
       return ARC_ERR_CUDA;
     d.attrs_set = true;
   }
@@ -108,17 +112,19 @@ int take_inject() {
 // ---------------------------------------------------------------------------------------------
 
 struct QuantWs {
-  uint32_t* amax;
+  uint32_t* partials;
   float* stash;
   double* inv_rms;
 };
 
+constexpr int64_t kPartialBytes = arc::kMaxPartials * 4;
+
 QuantWs carve_quant_ws(void* ws, int64_t rows, int32_t r) {
   uint8_t* b = static_cast<uint8_t*>(ws);
   QuantWs w;
-  w.amax = reinterpret_cast<uint32_t*>(b);
-  w.stash = reinterpret_cast<float*>(b + 256);
-  w.inv_rms = reinterpret_cast<double*>(b + 256 + align256(rows * static_cast<int64_t>(r) * 4));
+  w.partials = reinterpret_cast<uint32_t*>(b);
+  w.stash = reinterpret_cast<float*>(b + kPartialBytes);
+  w.inv_rms = reinterpret_cast<double*>(b + kPartialBytes + align256(rows * static_cast<int64_t>(r) * 4));
   return w;
 }
 
@@ -140,19 +146,22 @@ arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, con
   const double eps_d = static_cast<double>(eps);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   const __nv_bfloat16* gb = static_cast<const __nv_bfloat16*>(gain);
-  if (!static_scale) {
-    if (cudaMemsetAsync(w.amax, 0, 4, s) != cudaSuccess) return ARC_ERR_CUDA;
-  }
+  int npartials = 0;
   if (gain) {
-    arc::k_row_stats<<<static_cast<unsigned>((M + 7) / 8), 256, 0, s>>>(xb, ldx, static_cast<int>(M),
+    npartials = static_cast<int>(std::min<int64_t>((M + 7) / 8, arc::kMaxPartials));
+    arc::k_row_stats<<<static_cast<unsigned>(npartials), 256, 0, s>>>(xb, ldx, static_cast<int>(M),
                                                                      static_cast<int>(K), gb, eps_d, w.inv_rms,
-                                                                     static_scale ? nullptr : w.amax);
+                                                                     static_scale ? nullptr : w.partials);
   } else if (!static_scale) {
-    const int64_t vecs = M * (K / 8);
-    int64_t blocks = (vecs + 255) / 256;
-    blocks = std::min<int64_t>(blocks, static_cast<int64_t>(sms) * 8);
-    arc::k_amax<<<static_cast<unsigned>(std::max<int64_t>(blocks, 1)), 256, 0, s>>>(xb, ldx, static_cast<int>(M),
-                                                                                   static_cast<int>(K), w.amax);
+    if (ldx == K) {
+      const int64_t vecs = M * (K / 8);
+      npartials = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((vecs + 1023) / 1024, sms * 8)));
+      arc::k_amax<<<static_cast<unsigned>(npartials), 256, 0, s>>>(xb, vecs, w.partials);
+    } else {
+      npartials = static_cast<int>(std::min<int64_t>((M + 7) / 8, sms * 8));
+      arc::k_amax_rows<<<static_cast<unsigned>(npartials), 256, 0, s>>>(xb, ldx, static_cast<int>(M),
+                                                                        static_cast<int>(K), w.partials);
+    }
   }
   if ((st = launch_status()) != ARC_OK) return st;
   QuantArgs a;
@@ -167,14 +176,24 @@ arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, con
   a.gain = gb;
   a.inv_rms = w.inv_rms;
   a.static_scale = static_scale;
-  a.amax_word = w.amax;
+  a.partials = w.partials;
+  a.npartials = npartials;
   a.scale_out = scale_out;
   a.codes = codes;
   a.sf = sf;
   a.stash = w.stash;
   a.dup = dup;
-  dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>((K + 255) / 256));
-  arc::k_quant_main<<<grid, 256, 0, s>>>(a);
+  CUtensorMap tmx;
+  if (!make_map(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                static_cast<uint64_t>(ldx * 2), 64, 128))
+    return ARC_ERR_CUDA;
+  const int tiles_k = static_cast<int>((K + 127) / 128);
+  const int ntiles = static_cast<int>((M + 127) / 128) * tiles_k;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ntiles, static_cast<int64_t>(sms) * 3));
+  if (gain)
+    arc::k_quant_stream<true><<<grid, 256, arc::kQuantSmem, s>>>(tmx, a, tiles_k, ntiles, g_wait_ns);
+  else
+    arc::k_quant_stream<false><<<grid, 256, arc::kQuantSmem, s>>>(tmx, a, tiles_k, ntiles, g_wait_ns);
   if ((st = launch_status()) != ARC_OK) return st;
   if (a.kpad > a.K) {
     const int mpad = static_cast<int>((M + 127) / 128 * 128);
@@ -195,9 +214,9 @@ arc_status gemm_launch(const CUtensorMap& ta, const CUtensorMap& tb, GemmArgs g,
   const unsigned grid = static_cast<unsigned>(std::min(ntiles, sms));
   const int smem = arc::gemm_smem_bytes<FP4>();
   if (add)
-    arc::k_gemm<FP4, true><<<grid, 192, smem, s>>>(ta, tb, g);
+    arc::k_gemm<FP4, true><<<grid, arc::kGemmThreads, smem, s>>>(ta, tb, g);
   else
-    arc::k_gemm<FP4, false><<<grid, 192, smem, s>>>(ta, tb, g);
+    arc::k_gemm<FP4, false><<<grid, arc::kGemmThreads, smem, s>>>(ta, tb, g);
   return launch_status();
 }
 
@@ -236,7 +255,7 @@ size_t arc_nvfp4_sf_bytes(int64_t rows, int64_t k_aug) {
 
 size_t arc_quantize_workspace_bytes(int64_t rows, int32_t r) {
   if (rows < 0 || r < 0) return 0;
-  return static_cast<size_t>(256 + align256(rows * static_cast<int64_t>(r) * 4) + align256(rows * 8));
+  return static_cast<size_t>(kPartialBytes + align256(rows * static_cast<int64_t>(r) * 4) + align256(rows * 8));
 }
 
 size_t arc_calibrate_workspace_bytes(int64_t K) {

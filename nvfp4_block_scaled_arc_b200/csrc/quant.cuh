@@ -9,22 +9,28 @@
 // appended after the K primary channels.
 //
 // Work split:
-//   k_amax        whole-tensor max |x| (16-byte loads, integer max on |bf16| bit patterns,
-//                 one atomicMax per CTA) -> workspace word
-//   k_row_stats   one warp per row: exact sum of squares -> 1/rms (double), and with a dynamic
-//                 scale the max |RMSNorm(x)| as well
-//   k_quant_main  CTA tile 128 rows x 256 channels: 8 warps x 16 rows, one 16-byte load per
-//                 lane per row (a lane pair owns a block), codes stored as 4 bytes per lane
-//                 (128 contiguous bytes per warp), scale bytes staged in shared memory and
-//                 written as whole 512-byte atoms; outlier channels leave x (weights) or
-//                 x - deq (activations) in a [rows, r] fp32 stash
-//   k_quant_tail  one warp per row: the r/16 appended blocks from the stash plus zero padding
-//                 up to K_pad, including the zero scale bytes of padding rows
+//   k_amax        whole-tensor max |x|: 16-byte loads, 4 in flight per thread, integer max on
+//                 |bf16| bit patterns; one partial per CTA in the workspace (no atomics, no
+//                 initialisation of the workspace needed)
+//   k_row_stats   one warp per row: exact sum of squares -> 1/rms (double); with a dynamic
+//                 scale also max |RMSNorm(x)|, one partial per CTA
+//   k_quant_stream persistent CTAs over tiles of 128 rows x 128 channels, the X tile TMA-loaded
+//                 into shared memory (double-buffered); one lane per 16-element block (8 lanes
+//                 per row, 4 rows per warp step), packed-pair division, 8 code bytes per lane (a
+//                 row's 64 code bytes contiguous), scale bytes staged in shared memory and written
+//                 as whole 512-byte atoms; outlier channels leave x (weights) or x - deq
+//                 (activations) in a [rows, r] fp32 stash
+//   k_quant_tail  one warp per row: the r/16 appended blocks from the stash plus zero padding up
+//                 to K_pad, including the zero scale bytes of padding rows
+// Divisions are correctly rounded: x/d uses RN(1/d) and one exact-remainder correction
+// (Markstein), with a plain IEEE divide when an operand is outside [2^-90, 2^90].
 #pragma once
 
 #include "arc_device.cuh"
 
 namespace arc {
+
+constexpr int kMaxPartials = 2048;  // per-CTA abs-max partials at the start of the workspace
 
 struct QuantArgs {
   const __nv_bfloat16* x;
@@ -34,7 +40,8 @@ struct QuantArgs {
   const __nv_bfloat16* gain;  // RMSNorm prologue gain, or nullptr
   const double* inv_rms;      // [M] from k_row_stats when gain != nullptr
   const float* static_scale;  // or nullptr (dynamic)
-  const uint32_t* amax_word;  // fp32 bits of max |x| (dynamic)
+  const uint32_t* partials;   // fp32 bits of per-CTA max |x| (dynamic)
+  int npartials;
   float* scale_out;
   uint8_t* codes;
   uint8_t* sf;
@@ -50,9 +57,23 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   return v;
 }
 
-__device__ __forceinline__ float tensor_scale_of(const QuantArgs& a) {
+__device__ __forceinline__ bool in_safe_range(float v) {
+  return v >= 8.077935669463161e-28f && v <= 1.2379400392853803e27f;  // [2^-90, 2^90]
+}
+
+// Tensor scale of this call, by one CTA (all threads return the same value).
+__device__ float cta_tensor_scale(const QuantArgs& a) {
   if (a.static_scale) return *a.static_scale;
-  const float am = __uint_as_float(*a.amax_word);
+  __shared__ uint32_t red[32];
+  uint32_t mx = 0;
+  for (int i = threadIdx.x; i < a.npartials; i += blockDim.x) mx = max(mx, a.partials[i]);
+  mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  uint32_t b = 0;
+  for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) b = max(b, red[i]);
+  __syncthreads();
+  const float am = __uint_as_float(b);
   return am > 0.0f ? __fdiv_rn(am, 2688.0f) : 1.0f;
 }
 
@@ -61,30 +82,54 @@ __device__ __forceinline__ int64_t sf_offset(int64_t m, int64_t kb, int katoms) 
   return ((m >> 7) * katoms + (kb >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (kb & 3);
 }
 
-// Codes of up to 8 values against decode scale d (d > 0): E2M1 of the correctly rounded
-// quotient, sign bit taken from the value.
-__device__ __forceinline__ uint32_t encode8(const float (&v)[8], float d) {
-  float q[8];
-  if (d >= 7.888609052210118e-31f && d <= 1.2676506002282294e30f) {  // [2^-100, 2^100]
-    const float rcp = __frcp_rn(d);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) q[e] = div_rn_from_rcp(v[e], d, rcp);
+// Scale byte and decode scale d of a block with abs-max `amax` under tensor scale s:
+// t = (amax / 6) / s (two correctly rounded divides), sf = E4M3(t), d = E4M3value(sf) * s.
+__device__ __forceinline__ uint32_t block_scale(float amax, float s, float rcp_s, float rcp6, float* d) {
+  float t;
+  if (in_safe_range(amax) && in_safe_range(s)) {
+    const float t1 = div_rn_from_rcp(amax, 6.0f, rcp6);
+    const float q0 = __fmul_rn(t1, rcp_s);
+    // outside [2^-20, 2^20] the E4M3 result is 0 or 448 whatever the last bit of t
+    t = (q0 >= 9.5367431640625e-07f && q0 <= 1048576.0f) ? div_rn_from_rcp(t1, s, rcp_s) : q0;
   } else {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) q[e] = __fdiv_rn(v[e], d);
+    t = __fdiv_rn(__fdiv_rn(amax, 6.0f), s);
   }
-  uint32_t c = e2m1x8_rn_sat(q) & 0x77777777u;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) c |= (__float_as_uint(v[e]) >> 31) << (4 * e + 3);
-  return c;
-}
-
-// Scale byte and decode scale of a block with abs-max `amax` under tensor scale s.
-__device__ __forceinline__ uint32_t block_scale(float amax, float s, float* d) {
-  const float t = __fdiv_rn(__fdiv_rn(amax, 6.0f), s);
   const uint32_t sfb = e4m3_rn_sat(t);
   *d = __fmul_rn(e4m3_value(sfb), s);
   return sfb;
+}
+
+// Codes of 16 values (8 packed pairs) against decode scale d > 0: E2M1 of the correctly rounded
+// quotient. The hardware conversion keeps the sign of a quotient that rounds to zero (-0.1 ->
+// 0x8), so the sign bit follows x without extra work. Element i of pair j in bits 8j + 4i.
+__device__ __forceinline__ uint2 encode16(const uint64_t (&p)[8], float d) {
+  float q[16];
+  if (in_safe_range(d)) {
+    const float rcp = __frcp_rn(d);
+    const uint64_t rcp2 = f2_pack(rcp, rcp), nd2 = f2_pack(-d, -d);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      // the correction turns a -0 quotient into +0 ((+0) + (-0)); the quotient takes x's sign
+      const uint64_t qq = div2_rn_from_rcp(p[j], nd2, rcp2);
+      const uint64_t sg = 0x8000000080000000ull;
+      f2_unpack((qq & ~sg) | (p[j] & sg), q[2 * j], q[2 * j + 1]);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float x0, x1;
+      f2_unpack(p[j], x0, x1);
+      q[2 * j] = __fdiv_rn(x0, d);
+      q[2 * j + 1] = __fdiv_rn(x1, d);
+    }
+  }
+  float lo[8], hi[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    lo[i] = q[i];
+    hi[i] = q[8 + i];
+  }
+  return make_uint2(e2m1x8_rn_sat(lo), e2m1x8_rn_sat(hi));
 }
 
 // RMSNorm of one bf16 value: bf16( fp32( (h * inv) * g ) ), products in double.
@@ -93,57 +138,51 @@ __device__ __forceinline__ float rms_apply(float h, double inv, float g) {
   return __bfloat162float(__float2bfloat16_rn(__double2float_rn(t)));
 }
 
-// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t m, uint4 w) {
+  m = __vmaxu2(m, w.x & 0x7FFF7FFFu);
+  m = __vmaxu2(m, w.y & 0x7FFF7FFFu);
+  m = __vmaxu2(m, w.z & 0x7FFF7FFFu);
+  return __vmaxu2(m, w.w & 0x7FFF7FFFu);
+}
 
-__global__ void __launch_bounds__(256) k_amax(const __nv_bfloat16* __restrict__ x, int64_t ldx, int M, int K,
-                                              uint32_t* amax_word) {
-  const int vpr = K >> 3;  // 16-byte vectors per row
-  const int64_t total = static_cast<int64_t>(M) * vpr;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  uint32_t mx = 0;
-  int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (ldx == K) {
-    const uint4* p = reinterpret_cast<const uint4*>(x);
-    for (; v + 3 * stride < total; v += 4 * stride) {
-      uint4 w[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) w[u] = ld_nc_v4(p + v + u * stride);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        mx = __vmaxu2(mx, w[u].x & 0x7FFF7FFFu);
-        mx = __vmaxu2(mx, w[u].y & 0x7FFF7FFFu);
-        mx = __vmaxu2(mx, w[u].z & 0x7FFF7FFFu);
-        mx = __vmaxu2(mx, w[u].w & 0x7FFF7FFFu);
-      }
-    }
-    for (; v < total; v += stride) {
-      const uint4 w = ld_nc_v4(p + v);
-      mx = __vmaxu2(mx, w.x & 0x7FFF7FFFu);
-      mx = __vmaxu2(mx, w.y & 0x7FFF7FFFu);
-      mx = __vmaxu2(mx, w.z & 0x7FFF7FFFu);
-      mx = __vmaxu2(mx, w.w & 0x7FFF7FFFu);
-    }
-  } else {
-    for (; v < total; v += stride) {
-      const int64_t m = v / vpr, c = v - m * vpr;
-      const uint4 w = ld_nc_v4(x + m * ldx + 8 * c);
-      mx = __vmaxu2(mx, w.x & 0x7FFF7FFFu);
-      mx = __vmaxu2(mx, w.y & 0x7FFF7FFFu);
-      mx = __vmaxu2(mx, w.z & 0x7FFF7FFFu);
-      mx = __vmaxu2(mx, w.w & 0x7FFF7FFFu);
-    }
-  }
-  uint32_t m16 = max(mx & 0xFFFFu, mx >> 16);
-#pragma unroll
-  for (int o = 16; o; o >>= 1) m16 = max(m16, __shfl_xor_sync(0xFFFFFFFFu, m16, o));
-  __shared__ uint32_t red[8];
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m16;
+// Block-wide max of a per-thread value, written by thread 0 to *dst.
+__device__ __forceinline__ void cta_max_to(uint32_t v, uint32_t* dst) {
+  __shared__ uint32_t red[32];
+  v = __reduce_max_sync(0xFFFFFFFFu, v);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
   __syncthreads();
   if (threadIdx.x == 0) {
     uint32_t b = 0;
-    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) b = max(b, red[i]);
-    if (b) atomicMax(amax_word, b << 16);
+    for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) b = max(b, red[i]);
+    *dst = b;
   }
+}
+
+// ---------------------------------------------------------------------------------------------
+
+// Contiguous X (ldx == K): a flat stream of 16-byte vectors, 4 loads in flight per thread.
+__global__ void __launch_bounds__(256) k_amax(const __nv_bfloat16* __restrict__ x, int64_t nvec, uint32_t* partials) {
+  const uint4* p = reinterpret_cast<const uint4*>(x);
+  const int64_t T = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  uint32_t mx = 0;
+  int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; v + 3 * T < nvec; v += 4 * T) {
+    const uint4 w0 = ld_nc_v4(p + v), w1 = ld_nc_v4(p + v + T), w2 = ld_nc_v4(p + v + 2 * T),
+                w3 = ld_nc_v4(p + v + 3 * T);
+    mx = absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(mx, w0), w1), w2), w3);
+  }
+  for (; v < nvec; v += T) mx = absmax_bf16x2(mx, ld_nc_v4(p + v));
+  cta_max_to(max(mx & 0xFFFFu, mx >> 16) << 16, &partials[blockIdx.x]);
+}
+
+// Strided X (ldx > K): one row per warp-iteration.
+__global__ void __launch_bounds__(256) k_amax_rows(const __nv_bfloat16* __restrict__ x, int64_t ldx, int M, int K,
+                                                   uint32_t* partials) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t mx = 0;
+  for (int m = blockIdx.x * 8 + warp; m < M; m += gridDim.x * 8)
+    for (int k = 8 * lane; k < K; k += 256) mx = absmax_bf16x2(mx, ld_nc_v4(x + static_cast<int64_t>(m) * ldx + k));
+  cta_max_to(max(mx & 0xFFFFu, mx >> 16) << 16, &partials[blockIdx.x]);
 }
 
 // Round-to-nearest-even value of v * 2^e2 as a double (v < 2^128).
@@ -175,8 +214,7 @@ __device__ double warp_row_inv_rms(const __nv_bfloat16* __restrict__ h, int K, d
       if (b) emax = max(emax, max(static_cast<int>(b >> 7), 1));
     }
   }
-#pragma unroll
-  for (int o = 16; o; o >>= 1) emax = max(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, o));
+  emax = static_cast<int>(__reduce_max_sync(0xFFFFFFFFu, static_cast<unsigned>(emax)));
   unsigned __int128 acc = 0;
   for (int k = 8 * lane; k < K; k += 256) {
     const uint4 w = ld_nc_v4(h + k);
@@ -209,18 +247,18 @@ __device__ double warp_row_inv_rms(const __nv_bfloat16* __restrict__ h, int K, d
   return __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, static_cast<double>(K)), eps)));
 }
 
-// One warp per row: inv_rms[m]; with amax_word != nullptr also max |RMSNorm(h) * g|.
+// Warps over rows (grid-stride): inv_rms[m]; with partials != nullptr also max |RMSNorm(h)*g|,
+// one partial per CTA.
 __global__ void __launch_bounds__(256) k_row_stats(const __nv_bfloat16* __restrict__ h, int64_t ldh, int M, int K,
                                                    const __nv_bfloat16* __restrict__ gain, double eps,
-                                                   double* inv_rms, uint32_t* amax_word) {
+                                                   double* inv_rms, uint32_t* partials) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m = blockIdx.x * 8 + warp;
   uint32_t mx = 0;
-  if (m < M) {
+  for (int m = blockIdx.x * 8 + warp; m < M; m += gridDim.x * 8) {
     const __nv_bfloat16* row = h + static_cast<int64_t>(m) * ldh;
     const double inv = warp_row_inv_rms(row, K, eps, lane);
     if (lane == 0) inv_rms[m] = inv;
-    if (amax_word) {
+    if (partials) {
       for (int k = 8 * lane; k < K; k += 256) {
         const uint4 w = ld_nc_v4(row + k);
         const uint4 g = ld_nc_v4(gain + k);
@@ -234,101 +272,174 @@ __global__ void __launch_bounds__(256) k_row_stats(const __nv_bfloat16* __restri
       }
     }
   }
-  if (amax_word) {
-#pragma unroll
-    for (int o = 16; o; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-    if (lane == 0 && mx) atomicMax(amax_word, mx);
-  }
+  if (partials) cta_max_to(mx, &partials[blockIdx.x]);
 }
 
 // ---------------------------------------------------------------------------------------------
 
-__global__ void __launch_bounds__(256) k_quant_main(QuantArgs a) {
-  __shared__ __align__(16) uint32_t sf_tile[4 * 128];
-  __shared__ uint32_t omask[8];
-  __shared__ int16_t ocol[256];
+// Persistent, TMA-fed variant of the primary pass. Each CTA walks tiles t = blockIdx.x,
+// blockIdx.x + gridDim.x, ... of 128 rows x 128 channels; the X tile arrives in shared memory
+// as two TMA boxes of 64 channels with 128-byte swizzle (bank-conflict-free 16-byte reads),
+// double-buffered so the next tile loads while this one is coded. The tensor scale is reduced
+// from the abs-max partials while the first tiles are in flight.
+constexpr int kQTileBytes = 128 * 128 * 2;
+constexpr int kQuantSmem = 2 * kQTileBytes + 1024 + 1024;
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// Shared-memory byte address of 16-byte chunk `c` (0..15) of tile row `row` (two 64-channel
+// halves, each rows x 128 bytes with the 128-byte swizzle: chunk j of row r at (j ^ r%8) * 16).
+__device__ __forceinline__ uint32_t qtile_chunk(uint32_t base, int row, int c) {
+  const int h = c >> 3, j = c & 7;
+  return base + h * (128 * 128) + row * 128 + ((j ^ (row & 7)) << 4);
+}
+
+template <bool RMS>
+__global__ void __launch_bounds__(256) k_quant_stream(const __grid_constant__ CUtensorMap tmX, QuantArgs a,
+                                                      int tiles_k, int ntiles, uint64_t wait_ns) {
+  extern __shared__ uint8_t qsmem_raw[];
+  uint8_t* qs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsmem_raw) + 1023) & ~uintptr_t(1023));
+  uint32_t* sf_tile = reinterpret_cast<uint32_t*>(qs + 2 * kQTileBytes);
+  __shared__ uint64_t bar[2];
+  __shared__ uint32_t omask[4];
+  __shared__ int16_t ocol[128];
+  __shared__ int abort_sh;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int m0 = blockIdx.x * 128, k0 = blockIdx.y * 256;
-  for (int i = tid; i < 4 * 128; i += 256) sf_tile[i] = 0;
-  if (tid < 8) omask[tid] = 0;
-  __syncthreads();
-  for (int j = tid; j < a.r; j += 256) {
-    const int c = a.idx[j];
-    if (c >= k0 && c < k0 + 256) {
-      ocol[c - k0] = static_cast<int16_t>(j);
-      atomicOr(&omask[(c - k0) >> 5], 1u << ((c - k0) & 31));
-    }
-  }
-  const float s = tensor_scale_of(a);
-  if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *a.scale_out = s;
-  __syncthreads();
+  const uint32_t xbase = smem_u32(qs);
 
-  const int kcol = k0 + 8 * lane;
-  const bool colok = kcol < a.K;
-  const uint32_t obits = (omask[lane >> 2] >> ((lane & 3) * 8)) & 0xFFu;
-  float g[8];
-  if (a.gain) {
-    uint4 gw = make_uint4(0, 0, 0, 0);
-    if (colok) gw = ld_nc_v4(a.gain + kcol);
-    const uint32_t gs[4] = {gw.x, gw.y, gw.z, gw.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) g[i] = (i & 1) ? bf16_hi(gs[i >> 1]) : bf16_lo(gs[i >> 1]);
+  auto issue = [&](int t, int buf) {
+    const int tm = t / tiles_k, tk = t - (t / tiles_k) * tiles_k;
+    mbar_arrive_expect_tx(&bar[buf], kQTileBytes);
+    uint8_t* dst = qs + buf * kQTileBytes;
+    tma_load_2d(dst, &tmX, &bar[buf], tk * 128, tm * 128);
+    tma_load_2d(dst + 128 * 128, &tmX, &bar[buf], tk * 128 + 64, tm * 128);
+  };
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    abort_sh = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmX);
+    if (blockIdx.x < ntiles) issue(blockIdx.x, 0);
+    if (blockIdx.x + gridDim.x < ntiles) issue(blockIdx.x + gridDim.x, 1);
   }
-  uint8_t* sfb = reinterpret_cast<uint8_t*>(sf_tile);
-  const int blk = lane >> 1;  // block index inside the tile (0..15)
+  const float s = cta_tensor_scale(a);  // overlaps the first loads; contains __syncthreads
+  if (blockIdx.x == 0 && tid == 0) *a.scale_out = s;
+  const float rcp_s = __frcp_rn(s), rcp6 = __frcp_rn(6.0f);
+  const int b = lane & 7;      // block inside the tile
+  const int rsub = lane >> 3;  // row inside the warp's group of 4
   const int64_t cpitch = a.kpad >> 1;
+  uint8_t* sfb = reinterpret_cast<uint8_t*>(sf_tile);
 
-#pragma unroll 1
-  for (int i = 0; i < 16; i += 4) {
-    uint4 w[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int m = m0 + warp * 16 + i + u;
-      w[u] = make_uint4(0, 0, 0, 0);
-      if (m < a.M && colok) w[u] = ld_nc_v4(a.x + static_cast<int64_t>(m) * a.ldx + kcol);
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int mm = warp * 16 + i + u;  // row inside the tile
-      const int m = m0 + mm;
-      const uint32_t ws[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
-      float v[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = (e & 1) ? bf16_hi(ws[e >> 1]) : bf16_lo(ws[e >> 1]);
-      if (a.gain && m < a.M) {
-        const double inv = a.inv_rms[m];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = rms_apply(v[e], inv, g[e]);
+  int it = 0;
+  for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+    const int buf = it & 1;
+    const uint32_t par = (it >> 1) & 1;
+    const int tm = t / tiles_k, tk = t - tm * tiles_k;
+    const int m0 = tm * 128, k0 = tk * 128;
+    __syncthreads();  // the previous tile's scale atoms are written out
+    for (int i = tid; i < 256; i += 256) sf_tile[i] = 0;
+    if (tid < 4) omask[tid] = 0;
+    __syncthreads();
+    for (int j = tid; j < a.r; j += 256) {
+      const int c = a.idx[j];
+      if (c >= k0 && c < k0 + 128) {
+        ocol[c - k0] = static_cast<int16_t>(j);
+        atomicOr(&omask[(c - k0) >> 5], 1u << ((c - k0) & 31));
       }
-      float am = 0.0f;
+    }
+    // every thread waits for the tile; a wait that runs out stops the whole CTA
+    if (!mbar_wait(&bar[buf], par, wait_ns, &abort_sh)) abort_sh = 1;
+    __syncthreads();
+    if (abort_sh) break;
+
+    const int kcol = k0 + 16 * b;
+    const bool colok = kcol < a.K;
+    const uint32_t obits = (omask[b >> 1] >> ((b & 1) * 16)) & 0xFFFFu;
+    float g[16];
+    if (RMS) {
+      uint4 g0 = make_uint4(0, 0, 0, 0), g1 = g0;
+      if (colok) {
+        g0 = ld_nc_v4(a.gain + kcol);
+        g1 = ld_nc_v4(a.gain + kcol + 8);
+      }
+      const uint32_t gs[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
-      for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(v[e]));
-      am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
+      for (int i = 0; i < 16; ++i) g[i] = (i & 1) ? bf16_hi(gs[i >> 1]) : bf16_lo(gs[i >> 1]);
+    }
+    const uint32_t tbase = xbase + buf * kQTileBytes;
+#pragma unroll 1
+    for (int rg = 0; rg < 4; ++rg) {
+      const int mm = rg * 32 + warp * 4 + rsub;
+      const int m = m0 + mm;
+      const uint4 w0 = lds_v4(qtile_chunk(tbase, mm, 2 * b));
+      const uint4 w1 = lds_v4(qtile_chunk(tbase, mm, 2 * b + 1));
+      const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      uint64_t p[8];
+      float amax;
+      double inv = 0.0;
+      if (RMS) {
+        inv = (m < a.M) ? a.inv_rms[m] : 0.0;
+        float mx = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float v0 = rms_apply(bf16_lo(ws[j]), inv, g[2 * j]);
+          const float v1 = rms_apply(bf16_hi(ws[j]), inv, g[2 * j + 1]);
+          mx = fmaxf(mx, fmaxf(fabsf(v0), fabsf(v1)));
+          p[j] = f2_pack(v0, v1);
+        }
+        amax = mx;
+      } else {
+        uint32_t am2 = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          am2 = __vmaxu2(am2, ws[j] & 0x7FFF7FFFu);
+          p[j] = f2_pack(bf16_lo(ws[j]), bf16_hi(ws[j]));
+        }
+        amax = __uint_as_float(max(am2 & 0xFFFFu, am2 >> 16) << 16);
+      }
       float d;
-      const uint32_t sfv = block_scale(am, s, &d);
-      const uint32_t codes = (d == 0.0f) ? 0u : encode8(v, d);
+      const uint32_t sfv = block_scale(amax, s, rcp_s, rcp6, &d);
+      const uint2 codes = (d == 0.0f) ? make_uint2(0u, 0u) : encode16(p, d);
       if (m < a.M && colok) {
-        *reinterpret_cast<uint32_t*>(a.codes + static_cast<int64_t>(m) * cpitch + (kcol >> 1)) = codes;
-        if ((lane & 1) == 0) sfb[(blk >> 2) * 512 + (mm & 31) * 16 + (mm >> 5) * 4 + (blk & 3)] = static_cast<uint8_t>(sfv);
-        if (obits) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            if ((obits >> e) & 1u) {
-              const int j = ocol[8 * lane + e];
-              const float deq = __fmul_rn(e2m1_value((codes >> (4 * e)) & 15u), d);
-              a.stash[static_cast<int64_t>(m) * a.r + j] = a.dup ? v[e] : __fsub_rn(v[e], deq);
-            }
-          }
+        *reinterpret_cast<uint2*>(a.codes + static_cast<int64_t>(m) * cpitch + (kcol >> 1)) = codes;
+        sfb[(b >> 2) * 512 + (mm & 31) * 16 + (mm >> 5) * 4 + (b & 3)] = static_cast<uint8_t>(sfv);
+        uint32_t ob = obits;
+        while (ob) {
+          const int e = __ffs(ob) - 1;
+          ob &= ob - 1;
+          const uint32_t hv = *reinterpret_cast<const uint16_t*>(qs + buf * kQTileBytes +
+                                                                 (qtile_chunk(tbase, mm, 2 * b + (e >> 3)) - tbase) +
+                                                                 2 * (e & 7));
+          float v = __uint_as_float(hv << 16);
+          if (RMS) v = rms_apply(v, inv, __bfloat162float(a.gain[kcol + e]));
+          const uint32_t c = ((e < 8 ? codes.x : codes.y) >> (4 * (e & 7))) & 15u;
+          const float deq = __fmul_rn(e2m1_value(c), d);
+          a.stash[static_cast<int64_t>(m) * a.r + ocol[16 * b + e]] = a.dup ? v : __fsub_rn(v, deq);
         }
       }
     }
+    __syncthreads();  // tile buffer and scale staging complete
+    if (tid == 0 && t + 2 * static_cast<int>(gridDim.x) < ntiles) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      issue(t + 2 * gridDim.x, buf);
+    }
+    const int natoms = min(2, (a.K - k0 + 63) >> 6);
+    uint4* dst = reinterpret_cast<uint4*>(a.sf + (static_cast<int64_t>(tm) * a.katoms + (k0 >> 6)) * 512);
+    const uint4* src = reinterpret_cast<const uint4*>(sf_tile);
+    for (int i = tid; i < natoms * 32; i += 256) dst[i] = src[i];
   }
-  __syncthreads();
-  // whole atoms that hold primary blocks (a partly residual atom is finished by k_quant_tail)
-  const int natoms = min(4, (a.K - k0 + 63) >> 6);
-  uint4* dst = reinterpret_cast<uint4*>(a.sf + (static_cast<int64_t>(blockIdx.x) * a.katoms + (k0 >> 6)) * 512);
-  const uint4* src = reinterpret_cast<const uint4*>(sf_tile);
-  for (int t = tid; t < natoms * 32; t += 256) dst[t] = src[t];
+  // loads still in flight after an abort land before the CTA exits
+  if (tid == 0 && abort_sh) {
+    const uint64_t t0 = globaltimer_ns();
+    for (int i = 0; i < 2; ++i)
+      while (!mbar_test(&bar[(it + i) & 1], ((it + i) >> 1) & 1) && globaltimer_ns() - t0 < wait_ns) {
+      }
+  }
 }
 
 // One warp per row (rows up to the 128-padded count): appended residual blocks and padding.
@@ -337,31 +448,29 @@ __global__ void __launch_bounds__(256) k_quant_tail(QuantArgs a, int mpad) {
   const int m = blockIdx.x * 8 + warp;
   if (m >= mpad) return;
   const float s = (a.static_scale) ? *a.static_scale : *a.scale_out;
+  const float rcp_s = __frcp_rn(s), rcp6 = __frcp_rn(6.0f);
   const int nres = a.r >> 4;
   const int ntail = (a.kpad - a.K) >> 4;
   const int64_t cpitch = a.kpad >> 1;
   for (int b = lane; b < ntail; b += 32) {
-    uint32_t sfv = 0, c0 = 0, c1 = 0;
+    uint32_t sfv = 0;
+    uint2 codes = make_uint2(0u, 0u);
     if (m < a.M && b < nres) {
-      const float4* p = reinterpret_cast<const float4*>(a.stash + static_cast<int64_t>(m) * a.r + 16 * b);
-      float v0[8], v1[8];
-      const float4 q0 = p[0], q1 = p[1], q2 = p[2], q3 = p[3];
-      v0[0] = q0.x; v0[1] = q0.y; v0[2] = q0.z; v0[3] = q0.w;
-      v0[4] = q1.x; v0[5] = q1.y; v0[6] = q1.z; v0[7] = q1.w;
-      v1[0] = q2.x; v1[1] = q2.y; v1[2] = q2.z; v1[3] = q2.w;
-      v1[4] = q3.x; v1[5] = q3.y; v1[6] = q3.z; v1[7] = q3.w;
+      const float4* src = reinterpret_cast<const float4*>(a.stash + static_cast<int64_t>(m) * a.r + 16 * b);
+      uint64_t p[8];
       float am = 0.0f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) am = fmaxf(am, fmaxf(fabsf(v0[e]), fabsf(v1[e])));
-      float d;
-      sfv = block_scale(am, s, &d);
-      if (d != 0.0f) {
-        c0 = encode8(v0, d);
-        c1 = encode8(v1, d);
+      for (int i = 0; i < 4; ++i) {
+        const float4 q = src[i];
+        p[2 * i] = f2_pack(q.x, q.y);
+        p[2 * i + 1] = f2_pack(q.z, q.w);
+        am = fmaxf(am, fmaxf(fmaxf(fabsf(q.x), fabsf(q.y)), fmaxf(fabsf(q.z), fabsf(q.w))));
       }
+      float d;
+      sfv = block_scale(am, s, rcp_s, rcp6, &d);
+      if (d != 0.0f) codes = encode16(p, d);
     }
-    if (m < a.M)
-      *reinterpret_cast<uint2*>(a.codes + static_cast<int64_t>(m) * cpitch + ((a.K + 16 * b) >> 1)) = make_uint2(c0, c1);
+    if (m < a.M) *reinterpret_cast<uint2*>(a.codes + static_cast<int64_t>(m) * cpitch + ((a.K + 16 * b) >> 1)) = codes;
     a.sf[sf_offset(m, (a.K >> 4) + b, a.katoms)] = static_cast<uint8_t>(sfv);
   }
 }
