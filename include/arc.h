@@ -247,6 +247,39 @@ arc_status arc_set_wait_limit_ns(uint64_t ns);
  */
 arc_status arc_debug_inject(int32_t kind);
 
+/* ----------------------------------------------------------------------------------------- */
+/* Quantization without a workspace argument                                                  */
+/* ----------------------------------------------------------------------------------------- */
+
+/* Bytes of the fixed device array the call below uses (about 4.5 MiB). */
+#define ARC_STATIC_SCRATCH_BYTES 4726784
+
+/*
+ * The pages have no counterpart of this call: it changes where temporary memory comes from, not
+ * what is computed. It is for callers that cannot call cudaMalloc (or any allocator) while they
+ * run: a process that reserves all the device memory it will ever use when it starts and forbids
+ * allocation afterwards, or a plug-in hosted by a framework that owns the GPU's memory pool and
+ * gives its plug-ins no way to borrow from it. Such a caller cannot provide the workspace that
+ * arc_quantize_act_nvfp4 asks for.
+ *
+ * Same computation, arguments and outputs as arc_quantize_act_nvfp4 without `workspace` and
+ * `ws_bytes`; the call allocates nothing. Its temporary space is one array of
+ * ARC_STATIC_SCRATCH_BYTES bytes of device memory compiled into this library, so every GPU that
+ * loads the library holds that array until the process exits.
+ *   Limit: arc_quantize_workspace_bytes(M, r) <= ARC_STATIC_SCRATCH_BYTES (for example M = 4096
+ *          with r <= 256, or M = 16384 with r <= 64); larger requests return ARC_ERR_WORKSPACE
+ *          before any launch.
+ *   Set-up: the first call on a device looks up the array's device address on that device (it
+ *          must be the current device); make that first call before any stream capture.
+ *   Sharing: every call uses the same array and leaves its last contents in it; nothing in the
+ *          array needs to start at zero. Calls whose work overlaps on the GPU (other streams,
+ *          other host threads) race on the array and must be ordered by the caller.
+ */
+arc_status arc_quantize_act_nvfp4_static_scratch(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                                                 const int32_t* d_idx, int32_t r, const void* rms_gain_bf16,
+                                                 float rms_eps, const float* d_static_scale, uint8_t* codes,
+                                                 uint8_t* sf, float* d_scale_out, arc_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -80,6 +80,11 @@ _SIGS = {
     "arc_last_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "arc_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64]),
     "arc_debug_inject": (ctypes.c_int, [ctypes.c_int32]),
+    "arc_quantize_act_nvfp4_static_scratch": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                                             ctypes.c_int64, ctypes.c_void_p, ctypes.c_int32,
+                                                             ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p,
+                                                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                             ctypes.c_void_p]),
 }
 
 

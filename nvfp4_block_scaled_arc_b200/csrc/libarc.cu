@@ -515,6 +515,44 @@ arc_status arc_set_wait_limit_ns(uint64_t ns) {
   return ARC_OK;
 }
 
+}  // extern "C"
+
+// Temporary space of arc_quantize_act_nvfp4_static_scratch: one fixed array per device, for
+// callers that cannot allocate. Host code only ever passes the address that
+// cudaGetSymbolAddress returns for the current device, looked up once per device.
+static __device__ __align__(256) uint8_t g_static_scratch[ARC_STATIC_SCRATCH_BYTES];
+
+namespace {
+arc_status static_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ARC_ERR_CUDA;
+  static void* addr[64] = {};
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return ARC_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return ARC_OK;
+}
+}  // namespace
+
+extern "C" {
+
+arc_status arc_quantize_act_nvfp4_static_scratch(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                                                 const int32_t* d_idx, int32_t r, const void* rms_gain_bf16,
+                                                 float rms_eps, const float* d_static_scale, uint8_t* codes,
+                                                 uint8_t* sf, float* d_scale_out, arc_stream_t stream) {
+  if (M <= 0 || r < 0) return ARC_ERR_INVALID_ARG;
+  if (arc_quantize_workspace_bytes(M, r) > static_cast<size_t>(ARC_STATIC_SCRATCH_BYTES)) return ARC_ERR_WORKSPACE;
+  void* ws = nullptr;
+  const arc_status st = static_scratch_address(&ws);
+  if (st != ARC_OK) return st;
+  return quantize_common(x_bf16, M, K, ldx, d_idx, r, rms_gain_bf16, rms_eps, d_static_scale, codes, sf,
+                         d_scale_out, ws, ARC_STATIC_SCRATCH_BYTES, stream, 0);
+}
+
 arc_status arc_debug_inject(int32_t kind) {
   if (kind < 0 || kind > 1) return ARC_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lk(g_mu);
