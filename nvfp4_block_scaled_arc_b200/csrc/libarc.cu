@@ -3,6 +3,9 @@
 // Single translation unit: every kernel of the library is included here.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <atomic>
+#include <chrono>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -53,10 +56,10 @@ arc_status device_check(int* sms) {
                              arc::gemm_smem_bytes<false>()) != cudaSuccess ||
         cudaFuncSetAttribute(arc::k_gemm<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              arc::gemm_smem_bytes<false>()) != cudaSuccess ||
-        cudaFuncSetAttribute(arc::k_quant_stream<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             arc::kQuantSmem) != cudaSuccess ||
-        cudaFuncSetAttribute(arc::k_quant_stream<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             arc::kQuantSmem) != cudaSuccess)
+        cudaFuncSetAttribute(arc::k_quant_fused<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             arc::kFusedSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(arc::k_quant_fused<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             arc::kFusedSmem) != cudaSuccess)
       return ARC_ERR_CUDA;
     d.attrs_set = true;
   }
@@ -111,21 +114,35 @@ int take_inject() {
 // Quantization driver shared by activations and weights
 // ---------------------------------------------------------------------------------------------
 
+// Quantizer workspace: per-CTA abs-max partials | grid-barrier flags (two per CTA) | residual
+// stash [rows, r] fp32 | 1/rms per row (double). Nothing in it needs to be initialised.
 struct QuantWs {
   uint32_t* partials;
+  unsigned long long* flags;
   float* stash;
   double* inv_rms;
 };
 
 constexpr int64_t kPartialBytes = arc::kMaxPartials * 4;
+constexpr int64_t kFlagBytes = arc::kMaxPartials * 2 * 8;
 
 QuantWs carve_quant_ws(void* ws, int64_t rows, int32_t r) {
   uint8_t* b = static_cast<uint8_t*>(ws);
   QuantWs w;
   w.partials = reinterpret_cast<uint32_t*>(b);
-  w.stash = reinterpret_cast<float*>(b + kPartialBytes);
-  w.inv_rms = reinterpret_cast<double*>(b + kPartialBytes + align256(rows * static_cast<int64_t>(r) * 4));
+  w.flags = reinterpret_cast<unsigned long long*>(b + kPartialBytes);
+  w.stash = reinterpret_cast<float*>(b + kPartialBytes + kFlagBytes);
+  w.inv_rms =
+      reinterpret_cast<double*>(b + kPartialBytes + kFlagBytes + align256(rows * static_cast<int64_t>(r) * 4));
   return w;
+}
+
+// Barrier epochs: never reused within a process; the start is taken from the clock so that flags
+// left in recycled device memory by an earlier process do not match.
+unsigned long long next_epoch() {
+  static std::atomic<unsigned long long> counter{
+      (static_cast<unsigned long long>(std::chrono::steady_clock::now().time_since_epoch().count()) << 8) | 1ull};
+  return counter.fetch_add(2);
 }
 
 arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, const int32_t* idx, int32_t r,
@@ -148,22 +165,13 @@ arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, con
   const __nv_bfloat16* gb = static_cast<const __nv_bfloat16*>(gain);
   int npartials = 0;
   if (gain) {
+    // RMSNorm statistics (and, with a dynamic scale, the abs-max of the normalised rows) first
     npartials = static_cast<int>(std::min<int64_t>((M + 7) / 8, arc::kMaxPartials));
     arc::k_row_stats<<<static_cast<unsigned>(npartials), 256, 0, s>>>(xb, ldx, static_cast<int>(M),
                                                                      static_cast<int>(K), gb, eps_d, w.inv_rms,
                                                                      static_scale ? nullptr : w.partials);
-  } else if (!static_scale) {
-    if (ldx == K) {
-      const int64_t vecs = M * (K / 8);
-      npartials = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((vecs + 1023) / 1024, sms * 8)));
-      arc::k_amax<<<static_cast<unsigned>(npartials), 256, 0, s>>>(xb, vecs, w.partials);
-    } else {
-      npartials = static_cast<int>(std::min<int64_t>((M + 7) / 8, sms * 8));
-      arc::k_amax_rows<<<static_cast<unsigned>(npartials), 256, 0, s>>>(xb, ldx, static_cast<int>(M),
-                                                                        static_cast<int>(K), w.partials);
-    }
+    if ((st = launch_status()) != ARC_OK) return st;
   }
-  if ((st = launch_status()) != ARC_OK) return st;
   QuantArgs a;
   a.x = xb;
   a.ldx = ldx;
@@ -189,18 +197,30 @@ arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, con
     return ARC_ERR_CUDA;
   const int tiles_k = static_cast<int>((K + 127) / 128);
   const int ntiles = static_cast<int>((M + 127) / 128) * tiles_k;
-  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ntiles, static_cast<int64_t>(sms) * 3));
-  if (gain)
-    arc::k_quant_stream<true><<<grid, 256, arc::kQuantSmem, s>>>(tmx, a, tiles_k, ntiles, g_wait_ns);
-  else
-    arc::k_quant_stream<false><<<grid, 256, arc::kQuantSmem, s>>>(tmx, a, tiles_k, ntiles, g_wait_ns);
-  if ((st = launch_status()) != ARC_OK) return st;
-  if (a.kpad > a.K) {
-    const int mpad = static_cast<int>((M + 127) / 128 * 128);
-    arc::k_quant_tail<<<static_cast<unsigned>((mpad + 7) / 8), 256, 0, s>>>(a, mpad);
-    if ((st = launch_status()) != ARC_OK) return st;
-  }
-  return ARC_OK;
+  // one resident CTA per SM: the launch is cooperative, so every CTA runs at once and the grid
+  // barriers inside the kernel are safe
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gain ? arc::k_quant_fused<true> : arc::k_quant_fused<false>,
+                                                    arc::kFusedThreads, arc::kFusedSmem) != cudaSuccess ||
+      per_sm < 1)
+    return ARC_ERR_CUDA;
+  const int grid = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(ntiles), static_cast<int64_t>(sms) * per_sm,
+                                                        static_cast<int64_t>(arc::kMaxPartials)}));
+  arc::FusedArgs f;
+  f.tiles_k = tiles_k;
+  f.ntiles = ntiles;
+  f.do_amax = (!gain && !static_scale) ? 1 : 0;
+  f.partials = w.partials;
+  f.flags = w.flags;
+  f.epoch = next_epoch();
+  f.wait_ns = g_wait_ns;
+  f.mpad = static_cast<int>((M + 127) / 128 * 128);
+  void* args[] = {&tmx, &a, &f};
+  const cudaError_t e =
+      cudaLaunchCooperativeKernel(gain ? reinterpret_cast<const void*>(arc::k_quant_fused<true>)
+                                       : reinterpret_cast<const void*>(arc::k_quant_fused<false>),
+                                  dim3(grid), dim3(arc::kFusedThreads), args, arc::kFusedSmem, s);
+  return e == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -255,7 +275,8 @@ size_t arc_nvfp4_sf_bytes(int64_t rows, int64_t k_aug) {
 
 size_t arc_quantize_workspace_bytes(int64_t rows, int32_t r) {
   if (rows < 0 || r < 0) return 0;
-  return static_cast<size_t>(kPartialBytes + align256(rows * static_cast<int64_t>(r) * 4) + align256(rows * 8));
+  return static_cast<size_t>(kPartialBytes + kFlagBytes + align256(rows * static_cast<int64_t>(r) * 4) +
+                             align256(rows * 8));
 }
 
 size_t arc_calibrate_workspace_bytes(int64_t K) {

@@ -442,6 +442,309 @@ __global__ void __launch_bounds__(256) k_quant_stream(const __grid_constant__ CU
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Single-launch quantizer (cooperative launch, one CTA per SM, all CTAs resident).
+//   phase 1  (dynamic scale, no RMSNorm): stream the CTA's tiles through a ring of kFusedBufs
+//            shared-memory buffers, reduce max |x|, publish one partial per CTA;
+//   barrier  every CTA waits for every partial;
+//   phase 2  code the tiles: first those still resident in the ring, then the others, which
+//            stream through the ring again (mostly L2 hits);
+//   barrier  every residual value is in the stash;
+//   phase 3  the appended residual blocks and the padding, rows spread over all CTAs.
+// The grid barrier needs no initialised memory: each CTA stores the call's epoch (a number the
+// host never reuses) in its own flag and waits until every flag shows it, with the usual
+// time limit; a wait that runs out sets the status word and stops the CTA.
+// ---------------------------------------------------------------------------------------------
+constexpr int kFusedThreads = 512;
+constexpr int kFusedBufs = 6;
+constexpr int kFusedSmem = kFusedBufs * kQTileBytes + 1024 + 1024;
+
+__device__ __forceinline__ bool grid_barrier(volatile unsigned long long* flags, int G, unsigned long long epoch,
+                                             uint64_t wait_ns, int* abort_sh) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    flags[blockIdx.x] = epoch;
+  }
+  const uint64_t t0 = globaltimer_ns();
+  bool ok = true;
+  for (int i = threadIdx.x; i < G && ok; i += blockDim.x) {
+    while (flags[i] != epoch) {
+      if (globaltimer_ns() - t0 > wait_ns) {
+        ok = false;
+        break;
+      }
+      __nanosleep(64);
+    }
+  }
+  if (!ok) {
+    set_status(kStatusTimeout);
+    *reinterpret_cast<volatile int*>(abort_sh) = 1;
+  }
+  __threadfence();
+  __syncthreads();
+  return *reinterpret_cast<volatile int*>(abort_sh) == 0;
+}
+
+struct FusedArgs {
+  int tiles_k, ntiles;
+  int do_amax;                  // phase 1 runs (dynamic scale without RMSNorm)
+  uint32_t* partials;           // [gridDim.x] written by phase 1
+  unsigned long long* flags;    // [2 * gridDim.x] barrier flags
+  unsigned long long epoch;     // this call's barrier epochs: epoch and epoch + 1
+  uint64_t wait_ns;
+  int mpad;                     // rows rounded up to 128 (scale padding rows)
+};
+
+template <bool RMS>
+__device__ __forceinline__ void code_tile(const QuantArgs& a, const uint8_t* tile, uint32_t tbase, int tm, int tk,
+                                          float s, float rcp_s, float rcp6, uint32_t* sf_tile, uint32_t* omask,
+                                          int16_t* ocol) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m0 = tm * 128, k0 = tk * 128;
+  const int b = lane & 7, rsub = lane >> 3;
+  const int kcol = k0 + 16 * b;
+  const bool colok = kcol < a.K;
+  const uint32_t obits = (omask[b >> 1] >> ((b & 1) * 16)) & 0xFFFFu;
+  const int64_t cpitch = a.kpad >> 1;
+  uint8_t* sfb = reinterpret_cast<uint8_t*>(sf_tile);
+  float g[16];
+  if (RMS) {
+    uint4 g0 = make_uint4(0, 0, 0, 0), g1 = g0;
+    if (colok) {
+      g0 = ld_nc_v4(a.gain + kcol);
+      g1 = ld_nc_v4(a.gain + kcol + 8);
+    }
+    const uint32_t gs[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) g[i] = (i & 1) ? bf16_hi(gs[i >> 1]) : bf16_lo(gs[i >> 1]);
+  }
+  // 16 warps x 4 rows per step = 64 rows; two steps cover the 128-row tile
+#pragma unroll 1
+  for (int rg = 0; rg < 2; ++rg) {
+    const int mm = rg * 64 + warp * 4 + rsub;
+    const int m = m0 + mm;
+    const uint4 w0 = lds_v4(qtile_chunk(tbase, mm, 2 * b));
+    const uint4 w1 = lds_v4(qtile_chunk(tbase, mm, 2 * b + 1));
+    const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    uint64_t p[8];
+    float amax;
+    double inv = 0.0;
+    if (RMS) {
+      inv = (m < a.M) ? a.inv_rms[m] : 0.0;
+      float mx = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float v0 = rms_apply(bf16_lo(ws[j]), inv, g[2 * j]);
+        const float v1 = rms_apply(bf16_hi(ws[j]), inv, g[2 * j + 1]);
+        mx = fmaxf(mx, fmaxf(fabsf(v0), fabsf(v1)));
+        p[j] = f2_pack(v0, v1);
+      }
+      amax = mx;
+    } else {
+      uint32_t am2 = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        am2 = __vmaxu2(am2, ws[j] & 0x7FFF7FFFu);
+        p[j] = f2_pack(bf16_lo(ws[j]), bf16_hi(ws[j]));
+      }
+      amax = __uint_as_float(max(am2 & 0xFFFFu, am2 >> 16) << 16);
+    }
+    float d;
+    const uint32_t sfv = block_scale(amax, s, rcp_s, rcp6, &d);
+    const uint2 codes = (d == 0.0f) ? make_uint2(0u, 0u) : encode16(p, d);
+    if (m < a.M && colok) {
+      *reinterpret_cast<uint2*>(a.codes + static_cast<int64_t>(m) * cpitch + (kcol >> 1)) = codes;
+      sfb[(b >> 2) * 512 + (mm & 31) * 16 + (mm >> 5) * 4 + (b & 3)] = static_cast<uint8_t>(sfv);
+      uint32_t ob = obits;
+      while (ob) {
+        const int e = __ffs(ob) - 1;
+        ob &= ob - 1;
+        const uint32_t hv =
+            *reinterpret_cast<const uint16_t*>(tile + (qtile_chunk(tbase, mm, 2 * b + (e >> 3)) - tbase) + 2 * (e & 7));
+        float v = __uint_as_float(hv << 16);
+        if (RMS) v = rms_apply(v, inv, __bfloat162float(a.gain[kcol + e]));
+        const uint32_t c = ((e < 8 ? codes.x : codes.y) >> (4 * (e & 7))) & 15u;
+        const float deq = __fmul_rn(e2m1_value(c), d);
+        a.stash[static_cast<int64_t>(m) * a.r + ocol[16 * b + e]] = a.dup ? v : __fsub_rn(v, deq);
+      }
+    }
+  }
+}
+
+// The appended residual blocks (from the stash) and zero padding up to K_pad of one row.
+__device__ __forceinline__ void tail_row(const QuantArgs& a, int m, float s, float rcp_s, float rcp6, int lane) {
+  const int nres = a.r >> 4;
+  const int ntail = (a.kpad - a.K) >> 4;
+  const int64_t cpitch = a.kpad >> 1;
+  for (int b = lane; b < ntail; b += 32) {
+    uint32_t sfv = 0;
+    uint2 codes = make_uint2(0u, 0u);
+    if (m < a.M && b < nres) {
+      const float4* src = reinterpret_cast<const float4*>(a.stash + static_cast<int64_t>(m) * a.r + 16 * b);
+      uint64_t p[8];
+      float am = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 q = src[i];
+        p[2 * i] = f2_pack(q.x, q.y);
+        p[2 * i + 1] = f2_pack(q.z, q.w);
+        am = fmaxf(am, fmaxf(fmaxf(fabsf(q.x), fabsf(q.y)), fmaxf(fabsf(q.z), fabsf(q.w))));
+      }
+      float d;
+      sfv = block_scale(am, s, rcp_s, rcp6, &d);
+      if (d != 0.0f) codes = encode16(p, d);
+    }
+    if (m < a.M) *reinterpret_cast<uint2*>(a.codes + static_cast<int64_t>(m) * cpitch + ((a.K + 16 * b) >> 1)) = codes;
+    a.sf[sf_offset(m, (a.K >> 4) + b, a.katoms)] = static_cast<uint8_t>(sfv);
+  }
+}
+
+template <bool RMS>
+__global__ void __launch_bounds__(kFusedThreads, 1) k_quant_fused(const __grid_constant__ CUtensorMap tmX,
+                                                                  QuantArgs a, FusedArgs f) {
+  extern __shared__ uint8_t fsmem_raw[];
+  uint8_t* qs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fsmem_raw) + 1023) & ~uintptr_t(1023));
+  uint32_t* sf_tile = reinterpret_cast<uint32_t*>(qs + kFusedBufs * kQTileBytes);
+  __shared__ uint64_t bar[kFusedBufs];
+  __shared__ uint32_t omask[4];
+  __shared__ int16_t ocol[128];
+  __shared__ int abort_sh;
+  __shared__ int issued_sh;  // slots whose loads thread 0 has issued
+  __shared__ float s_sh;
+  const int tid = threadIdx.x;
+  const int G = gridDim.x;
+  const int n_c = (f.ntiles > static_cast<int>(blockIdx.x)) ? (f.ntiles - blockIdx.x + G - 1) / G : 0;
+  const uint32_t xbase = smem_u32(qs);
+  auto tile_of = [&](int i) { return static_cast<int>(blockIdx.x) + i * G; };  // CTA-local index -> tile
+  auto issue = [&](int slot, int i) {
+    const int t = tile_of(i);
+    const int tm = t / f.tiles_k, tk = t - (t / f.tiles_k) * f.tiles_k;
+    const int buf = slot % kFusedBufs;
+    mbar_arrive_expect_tx(&bar[buf], kQTileBytes);
+    uint8_t* dst = qs + buf * kQTileBytes;
+    tma_load_2d(dst, &tmX, &bar[buf], tk * 128, tm * 128);
+    tma_load_2d(dst + 128 * 128, &tmX, &bar[buf], tk * 128 + 64, tm * 128);
+    issued_sh = slot + 1;
+  };
+  auto wait_slot = [&](int slot) -> bool {
+    if (!mbar_wait(&bar[slot % kFusedBufs], static_cast<uint32_t>((slot / kFusedBufs) & 1), f.wait_ns, &abort_sh))
+      abort_sh = 1;
+    __syncthreads();
+    return abort_sh == 0;
+  };
+  // after an abort: let every load still in flight land (bounded) before the CTA exits
+  auto teardown = [&](int from_slot) {
+    if (tid == 0) {
+      const uint64_t t0 = globaltimer_ns();
+      for (int sl = from_slot; sl < issued_sh; ++sl)
+        while (!mbar_test(&bar[sl % kFusedBufs], static_cast<uint32_t>((sl / kFusedBufs) & 1)) &&
+               globaltimer_ns() - t0 < f.wait_ns) {
+        }
+    }
+  };
+  if (tid == 0) {
+    for (int i = 0; i < kFusedBufs; ++i) mbar_init(&bar[i], 1);
+    abort_sh = 0;
+    issued_sh = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmX);
+    for (int i = 0; i < min(n_c, kFusedBufs); ++i) issue(i, i);
+  }
+  __syncthreads();
+  int slot = 0;     // next slot to consume
+  int resident = 0;  // tiles left in the ring by phase 1 (CTA-local indices n_c-resident .. n_c-1)
+  if (f.do_amax) {
+    // ------------------------------------------------------------------ phase 1: max |x|
+    uint32_t mx = 0;
+    for (int i = 0; i < n_c; ++i, ++slot) {
+      if (!wait_slot(slot)) {
+        teardown(slot);
+        return;
+      }
+      const uint32_t tb = xbase + (slot % kFusedBufs) * kQTileBytes;
+      // 512 threads x 4 chunks of 16 bytes = the 32 KB tile
+#pragma unroll
+      for (int j = 0; j < 4; ++j) mx = absmax_bf16x2(mx, lds_v4(tb + (tid + j * kFusedThreads) * 16));
+      __syncthreads();
+      if (tid == 0 && i + kFusedBufs < n_c) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        issue(slot + kFusedBufs, i + kFusedBufs);
+      }
+    }
+    cta_max_to(max(mx & 0xFFFFu, mx >> 16) << 16, &f.partials[blockIdx.x]);
+    resident = min(n_c, kFusedBufs);
+    if (!grid_barrier(f.flags, G, f.epoch, f.wait_ns, &abort_sh)) return;
+  }
+  // ---------------------------------------------------------------------- phase 2: code tiles
+  {
+    QuantArgs aa = a;
+    if (f.do_amax) {
+      aa.partials = f.partials;
+      aa.npartials = G;
+    }
+    const float s = cta_tensor_scale(aa);
+    if (tid == 0) s_sh = s;
+  }
+  __syncthreads();
+  const float s = s_sh;
+  if (blockIdx.x == 0 && tid == 0) *a.scale_out = s;
+  const float rcp_s = __frcp_rn(s), rcp6 = __frcp_rn(6.0f);
+  // processing order: the resident tiles (slots n_c-resident .. n_c-1), then the rest
+  const int first_slot = f.do_amax ? n_c - resident : 0;
+  const int nproc = n_c;
+  for (int q = 0; q < nproc; ++q) {
+    const int cur = first_slot + q;  // slot of this tile
+    const int i = f.do_amax ? (q < resident ? n_c - resident + q : q - resident) : q;
+    const int t = tile_of(i);
+    const int tm = t / f.tiles_k, tk = t - tm * f.tiles_k;
+    const int k0 = tk * 128;
+    __syncthreads();
+    for (int j = tid; j < 256; j += kFusedThreads) sf_tile[j] = 0;
+    if (tid < 4) omask[tid] = 0;
+    __syncthreads();
+    for (int j = tid; j < a.r; j += kFusedThreads) {
+      const int c = a.idx[j];
+      if (c >= k0 && c < k0 + 128) {
+        ocol[c - k0] = static_cast<int16_t>(j);
+        atomicOr(&omask[(c - k0) >> 5], 1u << ((c - k0) & 31));
+      }
+    }
+    const bool loaded = f.do_amax && q < resident;  // already waited for in phase 1
+    if (!loaded) {
+      if (!wait_slot(cur)) {
+        teardown(cur);
+        return;
+      }
+    } else {
+      __syncthreads();
+    }
+    const int buf = cur % kFusedBufs;
+    code_tile<RMS>(a, qs + buf * kQTileBytes, xbase + buf * kQTileBytes, tm, tk, s, rcp_s, rcp6, sf_tile, omask,
+                   ocol);
+    __syncthreads();
+    // the next load into this buffer: the tile kFusedBufs slots later, if any
+    const int next = q + kFusedBufs;
+    if (tid == 0 && next < nproc) {
+      const int inext = f.do_amax ? (next < resident ? -1 : next - resident) : next;
+      if (inext >= 0) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        issue(cur + kFusedBufs, inext);
+      }
+    }
+    const int natoms = min(2, (a.K - k0 + 63) >> 6);
+    uint4* dst = reinterpret_cast<uint4*>(a.sf + (static_cast<int64_t>(tm) * a.katoms + (k0 >> 6)) * 512);
+    const uint4* src = reinterpret_cast<const uint4*>(sf_tile);
+    for (int j = tid; j < natoms * 32; j += kFusedThreads) dst[j] = src[j];
+  }
+  if (a.kpad == a.K) return;
+  // ---------------------------------------------------------------------- phase 3: tail
+  if (!grid_barrier(f.flags + G, G, f.epoch + 1, f.wait_ns, &abort_sh)) return;
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int m = blockIdx.x * (kFusedThreads / 32) + warp; m < f.mpad; m += G * (kFusedThreads / 32))
+    tail_row(a, m, s, rcp_s, rcp6, lane);
+}
+
 // One warp per row (rows up to the 128-padded count): appended residual blocks and padding.
 __global__ void __launch_bounds__(256) k_quant_tail(QuantArgs a, int mpad) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
