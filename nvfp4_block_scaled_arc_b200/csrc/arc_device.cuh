@@ -11,6 +11,7 @@
 namespace arc {
 
 // Status codes mirrored from arc.h (device code cannot include the C enum's header order).
+constexpr int kStatusInvalidArg = 1;
 constexpr int kStatusTimeout = 5;
 
 // Device status word of this library: the first error a kernel reports wins.
@@ -26,6 +27,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
+}
+
+// Release store / acquire load at GPU scope (grid-level flags between CTAs).
+__device__ __forceinline__ void st_release_gpu(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -292,11 +303,35 @@ __device__ __forceinline__ float div_rn_from_rcp(float x, float d, float rcp) {
   return __fmaf_rn(r, rcp, q);
 }
 
-// The same on a pair: x2 / d with nd2 = (-d, -d) and rcp2 = (RN(1/d), RN(1/d)).
-__device__ __forceinline__ uint64_t div2_rn_from_rcp(uint64_t x2, uint64_t nd2, uint64_t rcp2) {
-  const uint64_t q = f2_mul(x2, rcp2);
-  const uint64_t r = f2_fma(q, nd2, x2);
-  return f2_fma(r, rcp2, q);
+// The negated quotient of a pair, -(x2 / d), correctly rounded, from nrcp2 = (-RN(1/d), -RN(1/d))
+// and d2 = (d, d): q0 = RN(x * nrcp), rem = RN(d q0 + x) = x - d (-q0) exactly, and RN(rem nrcp
+// + q0). Working on the negated quotient keeps the sign of a zero quotient: x = -0 gives +0 and
+// x = +0 gives -0, where the plain correction would turn both into +0 ((+0) + (-0) = +0).
+__device__ __forceinline__ uint64_t neg_div2_rn(uint64_t x2, uint64_t d2, uint64_t nrcp2) {
+  const uint64_t q = f2_mul(x2, nrcp2);
+  const uint64_t r = f2_fma(d2, q, x2);
+  return f2_fma(r, nrcp2, q);
+}
+
+// max(|a|, |b|, |c|) in one sm_100 three-input max.
+__device__ __forceinline__ float fmax3_abs(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(fabsf(a)), "f"(fabsf(b)), "f"(fabsf(c)));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// E2M1 code of one fp32 value (round to nearest even, saturating, sign kept on zero).
+__device__ __forceinline__ uint32_t e2m1_rn_sat1(float q) {
+  uint16_t r;
+  asm("{\n\t.reg .b8 b0;\n\tcvt.rn.satfinite.e2m1x2.f32 b0, %1, %2;\n\tcvt.u16.u8 %0, b0;\n\t}"
+      : "=h"(r)
+      : "f"(0.0f), "f"(q));
+  return r & 0xFu;
 }
 
 }  // namespace arc

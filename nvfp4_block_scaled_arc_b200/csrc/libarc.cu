@@ -114,8 +114,9 @@ int take_inject() {
 // Quantization driver shared by activations and weights
 // ---------------------------------------------------------------------------------------------
 
-// Quantizer workspace: per-CTA abs-max partials | grid-barrier flags (two per CTA) | residual
-// stash [rows, r] fp32 | 1/rms per row (double). Nothing in it needs to be initialised.
+// Quantizer workspace: per-CTA abs-max partials | grid-barrier words (two go words, two arrival
+// words per CTA) | residual stash [r, rows] fp32 | 1/rms per row (double). Nothing in it needs
+// to be initialised.
 struct QuantWs {
   uint32_t* partials;
   unsigned long long* flags;
@@ -204,8 +205,9 @@ arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, con
                                                     arc::kFusedThreads, arc::kFusedSmem) != cudaSuccess ||
       per_sm < 1)
     return ARC_ERR_CUDA;
+  // the barrier words hold two go words (256 bytes) and two arrival words per CTA
   const int grid = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(ntiles), static_cast<int64_t>(sms) * per_sm,
-                                                        static_cast<int64_t>(arc::kMaxPartials)}));
+                                                        static_cast<int64_t>(arc::kMaxPartials - 16)}));
   arc::FusedArgs f;
   f.tiles_k = tiles_k;
   f.ntiles = ntiles;

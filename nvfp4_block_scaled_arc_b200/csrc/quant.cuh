@@ -1,29 +1,35 @@
-// quant.cuh -- the memory-bound half of the hot path: tensor abs-max, RMSNorm statistics,
-// fused primary NVFP4 quantization with the residual stash, and the residual-channel tail.
+// quant.cuh -- the memory-bound half of the hot path: RMSNorm statistics and the single-launch
+// NVFP4 quantizer with its augmented residual channels.
 //
 // Method ("ARCQuant: Boosting NVFP4 Quantization with Augmented Residual Channels for LLMs",
 // Methodologie, Dual-Stage Quantisatie / Kernel Implementatie; "Day 0 LLM Inference Support",
 // section V items 1, 2 and 4): per 16-element block sf = E4M3((amax/6)/s), d = E4M3(sf)*s,
 // code = E2M1(x/d) with the sign of x, all-zero blocks give sf 0 and codes 0; the residual of
 // each outlier channel, x - E2M1(code)*d, is quantized again with the same tensor scale and
-// appended after the K primary channels.
+// appended after the K primary channels (weights append the channel itself).
 //
 // Work split:
-//   k_amax        whole-tensor max |x|: 16-byte loads, 4 in flight per thread, integer max on
-//                 |bf16| bit patterns; one partial per CTA in the workspace (no atomics, no
-//                 initialisation of the workspace needed)
-//   k_row_stats   one warp per row: exact sum of squares -> 1/rms (double); with a dynamic
-//                 scale also max |RMSNorm(x)|, one partial per CTA
-//   k_quant_stream persistent CTAs over tiles of 128 rows x 128 channels, the X tile TMA-loaded
-//                 into shared memory (double-buffered); one lane per 16-element block (8 lanes
-//                 per row, 4 rows per warp step), packed-pair division, 8 code bytes per lane (a
-//                 row's 64 code bytes contiguous), scale bytes staged in shared memory and written
-//                 as whole 512-byte atoms; outlier channels leave x (weights) or x - deq
-//                 (activations) in a [rows, r] fp32 stash
-//   k_quant_tail  one warp per row: the r/16 appended blocks from the stash plus zero padding up
-//                 to K_pad, including the zero scale bytes of padding rows
-// Divisions are correctly rounded: x/d uses RN(1/d) and one exact-remainder correction
-// (Markstein), with a plain IEEE divide when an operand is outside [2^-90, 2^90].
+//   k_row_stats    one warp per row: exact sum of squares -> 1/rms (double); with a dynamic
+//                  scale also max |RMSNorm(x)|, one partial per CTA
+//   k_quant_fused  one cooperative launch, one CTA per SM, tiles of 128 rows x 128 channels
+//                  TMA-loaded into a ring of shared-memory buffers by a producer warp, which
+//                  also lists each tile's outlier channels; sixteen coding warps take the tiles
+//                  (full/empty mbarriers between the two roles):
+//     phase 1  (dynamic scale without RMSNorm) max |x| over the CTA's tiles, the last ones
+//              staying resident in the ring; grid barrier; every CTA reduces the partials
+//     phase 2  code the tiles (resident ones first): each coding warp takes eight rows of a
+//              tile, one lane per 16-element block; codes and scale bytes go straight to
+//              global memory; then the warp stashes the residuals of the outlier channels
+//              of its rows in the column-major stash [r, M] (one (row, outlier) pair per
+//              lane, operands fetched by warp shuffles); the warps never wait for one
+//              another, only for tiles
+//     phase 3  after a second grid barrier: the appended residual blocks and the zero
+//              padding up to K_pad, one lane per (row, block) with rows fastest, so the
+//              stash reads are coalesced
+// Divisions are correctly rounded: x/d is formed as the negated quotient from -RN(1/d) with one
+// exact-remainder correction (Markstein), which keeps the sign of zero quotients, and the codes
+// of the negated quotients have their sign bits flipped back; a plain IEEE divide is used when
+// an operand is outside [2^-90, 2^90].
 #pragma once
 
 #include "arc_device.cuh"
@@ -45,7 +51,7 @@ struct QuantArgs {
   float* scale_out;
   uint8_t* codes;
   uint8_t* sf;
-  float* stash;  // [M, r]
+  float* stash;  // [r, M]: column j holds channel idx[j] of every row
   int dup;       // 1: weights (stash the value itself), 0: activations (stash the residual)
 };
 
@@ -54,6 +60,12 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
   return v;
 }
 
@@ -100,36 +112,33 @@ __device__ __forceinline__ uint32_t block_scale(float amax, float s, float rcp_s
 }
 
 // Codes of 16 values (8 packed pairs) against decode scale d > 0: E2M1 of the correctly rounded
-// quotient. The hardware conversion keeps the sign of a quotient that rounds to zero (-0.1 ->
-// 0x8), so the sign bit follows x without extra work. Element i of pair j in bits 8j + 4i.
+// quotient with the sign of x (a quotient that rounds to zero keeps it: -0.1 -> 0x8). The
+// quotients are formed negated, which keeps signed zeros exact, and since E2M1 is sign-magnitude
+// with symmetric rounding and saturation, code(q) = code(-q) ^ 8 nibble by nibble. Element i of
+// pair j in bits 8j + 4i.
 __device__ __forceinline__ uint2 encode16(const uint64_t (&p)[8], float d) {
-  float q[16];
+  float nq[16];
   if (in_safe_range(d)) {
-    const float rcp = __frcp_rn(d);
-    const uint64_t rcp2 = f2_pack(rcp, rcp), nd2 = f2_pack(-d, -d);
+    const float nrcp = -__frcp_rn(d);
+    const uint64_t nrcp2 = f2_pack(nrcp, nrcp), d2 = f2_pack(d, d);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      // the correction turns a -0 quotient into +0 ((+0) + (-0)); the quotient takes x's sign
-      const uint64_t qq = div2_rn_from_rcp(p[j], nd2, rcp2);
-      const uint64_t sg = 0x8000000080000000ull;
-      f2_unpack((qq & ~sg) | (p[j] & sg), q[2 * j], q[2 * j + 1]);
-    }
+    for (int j = 0; j < 8; ++j) f2_unpack(neg_div2_rn(p[j], d2, nrcp2), nq[2 * j], nq[2 * j + 1]);
   } else {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       float x0, x1;
       f2_unpack(p[j], x0, x1);
-      q[2 * j] = __fdiv_rn(x0, d);
-      q[2 * j + 1] = __fdiv_rn(x1, d);
+      nq[2 * j] = -__fdiv_rn(x0, d);
+      nq[2 * j + 1] = -__fdiv_rn(x1, d);
     }
   }
   float lo[8], hi[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    lo[i] = q[i];
-    hi[i] = q[8 + i];
+    lo[i] = nq[i];
+    hi[i] = nq[8 + i];
   }
-  return make_uint2(e2m1x8_rn_sat(lo), e2m1x8_rn_sat(hi));
+  return make_uint2(e2m1x8_rn_sat(lo) ^ 0x88888888u, e2m1x8_rn_sat(hi) ^ 0x88888888u);
 }
 
 // RMSNorm of one bf16 value: bf16( fp32( (h * inv) * g ) ), products in double.
@@ -159,31 +168,6 @@ __device__ __forceinline__ void cta_max_to(uint32_t v, uint32_t* dst) {
 }
 
 // ---------------------------------------------------------------------------------------------
-
-// Contiguous X (ldx == K): a flat stream of 16-byte vectors, 4 loads in flight per thread.
-__global__ void __launch_bounds__(256) k_amax(const __nv_bfloat16* __restrict__ x, int64_t nvec, uint32_t* partials) {
-  const uint4* p = reinterpret_cast<const uint4*>(x);
-  const int64_t T = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  uint32_t mx = 0;
-  int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  for (; v + 3 * T < nvec; v += 4 * T) {
-    const uint4 w0 = ld_nc_v4(p + v), w1 = ld_nc_v4(p + v + T), w2 = ld_nc_v4(p + v + 2 * T),
-                w3 = ld_nc_v4(p + v + 3 * T);
-    mx = absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(mx, w0), w1), w2), w3);
-  }
-  for (; v < nvec; v += T) mx = absmax_bf16x2(mx, ld_nc_v4(p + v));
-  cta_max_to(max(mx & 0xFFFFu, mx >> 16) << 16, &partials[blockIdx.x]);
-}
-
-// Strided X (ldx > K): one row per warp-iteration.
-__global__ void __launch_bounds__(256) k_amax_rows(const __nv_bfloat16* __restrict__ x, int64_t ldx, int M, int K,
-                                                   uint32_t* partials) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint32_t mx = 0;
-  for (int m = blockIdx.x * 8 + warp; m < M; m += gridDim.x * 8)
-    for (int k = 8 * lane; k < K; k += 256) mx = absmax_bf16x2(mx, ld_nc_v4(x + static_cast<int64_t>(m) * ldx + k));
-  cta_max_to(max(mx & 0xFFFFu, mx >> 16) << 16, &partials[blockIdx.x]);
-}
 
 // Round-to-nearest-even value of v * 2^e2 as a double (v < 2^128).
 __device__ __forceinline__ double u128_scaled_to_double(unsigned __int128 v, int e2) {
@@ -276,212 +260,55 @@ __global__ void __launch_bounds__(256) k_row_stats(const __nv_bfloat16* __restri
 }
 
 // ---------------------------------------------------------------------------------------------
-
-// Persistent, TMA-fed variant of the primary pass. Each CTA walks tiles t = blockIdx.x,
-// blockIdx.x + gridDim.x, ... of 128 rows x 128 channels; the X tile arrives in shared memory
-// as two TMA boxes of 64 channels with 128-byte swizzle (bank-conflict-free 16-byte reads),
-// double-buffered so the next tile loads while this one is coded. The tensor scale is reduced
-// from the abs-max partials while the first tiles are in flight.
-constexpr int kQTileBytes = 128 * 128 * 2;
-constexpr int kQuantSmem = 2 * kQTileBytes + 1024 + 1024;
-
-__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
-
-// Shared-memory byte address of 16-byte chunk `c` (0..15) of tile row `row` (two 64-channel
-// halves, each rows x 128 bytes with the 128-byte swizzle: chunk j of row r at (j ^ r%8) * 16).
-__device__ __forceinline__ uint32_t qtile_chunk(uint32_t base, int row, int c) {
-  const int h = c >> 3, j = c & 7;
-  return base + h * (128 * 128) + row * 128 + ((j ^ (row & 7)) << 4);
-}
-
-template <bool RMS>
-__global__ void __launch_bounds__(256) k_quant_stream(const __grid_constant__ CUtensorMap tmX, QuantArgs a,
-                                                      int tiles_k, int ntiles, uint64_t wait_ns) {
-  extern __shared__ uint8_t qsmem_raw[];
-  uint8_t* qs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsmem_raw) + 1023) & ~uintptr_t(1023));
-  uint32_t* sf_tile = reinterpret_cast<uint32_t*>(qs + 2 * kQTileBytes);
-  __shared__ uint64_t bar[2];
-  __shared__ uint32_t omask[4];
-  __shared__ int16_t ocol[128];
-  __shared__ int abort_sh;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t xbase = smem_u32(qs);
-
-  auto issue = [&](int t, int buf) {
-    const int tm = t / tiles_k, tk = t - (t / tiles_k) * tiles_k;
-    mbar_arrive_expect_tx(&bar[buf], kQTileBytes);
-    uint8_t* dst = qs + buf * kQTileBytes;
-    tma_load_2d(dst, &tmX, &bar[buf], tk * 128, tm * 128);
-    tma_load_2d(dst + 128 * 128, &tmX, &bar[buf], tk * 128 + 64, tm * 128);
-  };
-  if (tid == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
-    abort_sh = 0;
-    fence_mbar_init();
-    tma_prefetch_desc(&tmX);
-    if (blockIdx.x < ntiles) issue(blockIdx.x, 0);
-    if (blockIdx.x + gridDim.x < ntiles) issue(blockIdx.x + gridDim.x, 1);
-  }
-  const float s = cta_tensor_scale(a);  // overlaps the first loads; contains __syncthreads
-  if (blockIdx.x == 0 && tid == 0) *a.scale_out = s;
-  const float rcp_s = __frcp_rn(s), rcp6 = __frcp_rn(6.0f);
-  const int b = lane & 7;      // block inside the tile
-  const int rsub = lane >> 3;  // row inside the warp's group of 4
-  const int64_t cpitch = a.kpad >> 1;
-  uint8_t* sfb = reinterpret_cast<uint8_t*>(sf_tile);
-
-  int it = 0;
-  for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
-    const int buf = it & 1;
-    const uint32_t par = (it >> 1) & 1;
-    const int tm = t / tiles_k, tk = t - tm * tiles_k;
-    const int m0 = tm * 128, k0 = tk * 128;
-    __syncthreads();  // the previous tile's scale atoms are written out
-    for (int i = tid; i < 256; i += 256) sf_tile[i] = 0;
-    if (tid < 4) omask[tid] = 0;
-    __syncthreads();
-    for (int j = tid; j < a.r; j += 256) {
-      const int c = a.idx[j];
-      if (c >= k0 && c < k0 + 128) {
-        ocol[c - k0] = static_cast<int16_t>(j);
-        atomicOr(&omask[(c - k0) >> 5], 1u << ((c - k0) & 31));
-      }
-    }
-    // every thread waits for the tile; a wait that runs out stops the whole CTA
-    if (!mbar_wait(&bar[buf], par, wait_ns, &abort_sh)) abort_sh = 1;
-    __syncthreads();
-    if (abort_sh) break;
-
-    const int kcol = k0 + 16 * b;
-    const bool colok = kcol < a.K;
-    const uint32_t obits = (omask[b >> 1] >> ((b & 1) * 16)) & 0xFFFFu;
-    float g[16];
-    if (RMS) {
-      uint4 g0 = make_uint4(0, 0, 0, 0), g1 = g0;
-      if (colok) {
-        g0 = ld_nc_v4(a.gain + kcol);
-        g1 = ld_nc_v4(a.gain + kcol + 8);
-      }
-      const uint32_t gs[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-#pragma unroll
-      for (int i = 0; i < 16; ++i) g[i] = (i & 1) ? bf16_hi(gs[i >> 1]) : bf16_lo(gs[i >> 1]);
-    }
-    const uint32_t tbase = xbase + buf * kQTileBytes;
-#pragma unroll 1
-    for (int rg = 0; rg < 4; ++rg) {
-      const int mm = rg * 32 + warp * 4 + rsub;
-      const int m = m0 + mm;
-      const uint4 w0 = lds_v4(qtile_chunk(tbase, mm, 2 * b));
-      const uint4 w1 = lds_v4(qtile_chunk(tbase, mm, 2 * b + 1));
-      const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-      uint64_t p[8];
-      float amax;
-      double inv = 0.0;
-      if (RMS) {
-        inv = (m < a.M) ? a.inv_rms[m] : 0.0;
-        float mx = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float v0 = rms_apply(bf16_lo(ws[j]), inv, g[2 * j]);
-          const float v1 = rms_apply(bf16_hi(ws[j]), inv, g[2 * j + 1]);
-          mx = fmaxf(mx, fmaxf(fabsf(v0), fabsf(v1)));
-          p[j] = f2_pack(v0, v1);
-        }
-        amax = mx;
-      } else {
-        uint32_t am2 = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          am2 = __vmaxu2(am2, ws[j] & 0x7FFF7FFFu);
-          p[j] = f2_pack(bf16_lo(ws[j]), bf16_hi(ws[j]));
-        }
-        amax = __uint_as_float(max(am2 & 0xFFFFu, am2 >> 16) << 16);
-      }
-      float d;
-      const uint32_t sfv = block_scale(amax, s, rcp_s, rcp6, &d);
-      const uint2 codes = (d == 0.0f) ? make_uint2(0u, 0u) : encode16(p, d);
-      if (m < a.M && colok) {
-        *reinterpret_cast<uint2*>(a.codes + static_cast<int64_t>(m) * cpitch + (kcol >> 1)) = codes;
-        sfb[(b >> 2) * 512 + (mm & 31) * 16 + (mm >> 5) * 4 + (b & 3)] = static_cast<uint8_t>(sfv);
-        uint32_t ob = obits;
-        while (ob) {
-          const int e = __ffs(ob) - 1;
-          ob &= ob - 1;
-          const uint32_t hv = *reinterpret_cast<const uint16_t*>(qs + buf * kQTileBytes +
-                                                                 (qtile_chunk(tbase, mm, 2 * b + (e >> 3)) - tbase) +
-                                                                 2 * (e & 7));
-          float v = __uint_as_float(hv << 16);
-          if (RMS) v = rms_apply(v, inv, __bfloat162float(a.gain[kcol + e]));
-          const uint32_t c = ((e < 8 ? codes.x : codes.y) >> (4 * (e & 7))) & 15u;
-          const float deq = __fmul_rn(e2m1_value(c), d);
-          a.stash[static_cast<int64_t>(m) * a.r + ocol[16 * b + e]] = a.dup ? v : __fsub_rn(v, deq);
-        }
-      }
-    }
-    __syncthreads();  // tile buffer and scale staging complete
-    if (tid == 0 && t + 2 * static_cast<int>(gridDim.x) < ntiles) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      issue(t + 2 * gridDim.x, buf);
-    }
-    const int natoms = min(2, (a.K - k0 + 63) >> 6);
-    uint4* dst = reinterpret_cast<uint4*>(a.sf + (static_cast<int64_t>(tm) * a.katoms + (k0 >> 6)) * 512);
-    const uint4* src = reinterpret_cast<const uint4*>(sf_tile);
-    for (int i = tid; i < natoms * 32; i += 256) dst[i] = src[i];
-  }
-  // loads still in flight after an abort land before the CTA exits
-  if (tid == 0 && abort_sh) {
-    const uint64_t t0 = globaltimer_ns();
-    for (int i = 0; i < 2; ++i)
-      while (!mbar_test(&bar[(it + i) & 1], ((it + i) >> 1) & 1) && globaltimer_ns() - t0 < wait_ns) {
-      }
-  }
-}
-
-// ---------------------------------------------------------------------------------------------
 // Single-launch quantizer (cooperative launch, one CTA per SM, all CTAs resident).
-//   phase 1  (dynamic scale, no RMSNorm): stream the CTA's tiles through a ring of kFusedBufs
-//            shared-memory buffers, reduce max |x|, publish one partial per CTA;
-//   barrier  every CTA waits for every partial;
-//   phase 2  code the tiles: first those still resident in the ring, then the others, which
-//            stream through the ring again (mostly L2 hits);
-//   barrier  every residual value is in the stash;
-//   phase 3  the appended residual blocks and the padding, rows spread over all CTAs.
-// The grid barrier needs no initialised memory: each CTA stores the call's epoch (a number the
-// host never reuses) in its own flag and waits until every flag shows it, with the usual
-// time limit; a wait that runs out sets the status word and stops the CTA.
+// The grid barriers need no initialised memory: each CTA stores the call's epoch (a number the
+// host never reuses) in its own flag and waits until every flag shows it, with the usual time
+// limit; a wait that runs out sets the status word and stops the CTA.
 // ---------------------------------------------------------------------------------------------
-constexpr int kFusedThreads = 512;
+constexpr int kQTileBytes = 128 * 128 * 2;  // one X tile: two TMA boxes of 128 rows x 64 channels
+constexpr int kCodeWarps = 16;                      // warps that code tiles
+constexpr int kFusedThreads = (kCodeWarps + 1) * 32;  // plus one producer warp (loads, outlier lists)
 constexpr int kFusedBufs = 6;
-constexpr int kFusedSmem = kFusedBufs * kQTileBytes + 1024 + 1024;
+constexpr int kIdxSmem = 1024;  // outlier indices kept in shared memory (the rest read from L2)
+// dynamic shared memory: the ring of X tiles, 1024-aligned for the 128-byte swizzle
+constexpr int kFusedSmem = 1024 + kFusedBufs * kQTileBytes;
 
-__device__ __forceinline__ bool grid_barrier(volatile unsigned long long* flags, int G, unsigned long long epoch,
-                                             uint64_t wait_ns, int* abort_sh) {
+// Grid barrier over co-resident CTAs: each CTA publishes the call's epoch in its own arrival
+// word; CTA 0 gathers them (one polling thread per word) and then publishes the epoch in the
+// go word, which one thread of every CTA polls. Polling from every CTA on every arrival word
+// crowds a few L2 lines with requests and costs about twice as much. Release stores and acquire
+// loads at GPU scope carry each CTA's earlier writes (made visible to thread 0 by the CTA
+// barrier) to every CTA after the barrier. Every wait is bounded; one that runs out sets the
+// status word and makes the barrier return false in every CTA that sees it.
+__device__ __forceinline__ bool grid_barrier(unsigned long long* arrive, unsigned long long* go, int G,
+                                             unsigned long long epoch, uint64_t wait_ns, int* abort_sh) {
   __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    flags[blockIdx.x] = epoch;
-  }
+  if (threadIdx.x == 0) st_release_gpu(&arrive[blockIdx.x], epoch);
   const uint64_t t0 = globaltimer_ns();
   bool ok = true;
-  for (int i = threadIdx.x; i < G && ok; i += blockDim.x) {
-    while (flags[i] != epoch) {
+  if (blockIdx.x == 0) {
+    for (int i = threadIdx.x; i < G && ok; i += blockDim.x)
+      while (ld_acquire_gpu(&arrive[i]) != epoch) {
+        if (globaltimer_ns() - t0 > wait_ns) {
+          ok = false;
+          break;
+        }
+      }
+    ok = __syncthreads_and(ok);
+    if (threadIdx.x == 0 && ok) st_release_gpu(go, epoch);
+  }
+  if (threadIdx.x == 0 && ok) {
+    while (ld_acquire_gpu(go) != epoch) {
       if (globaltimer_ns() - t0 > wait_ns) {
         ok = false;
         break;
       }
-      __nanosleep(64);
     }
   }
   if (!ok) {
     set_status(kStatusTimeout);
     *reinterpret_cast<volatile int*>(abort_sh) = 1;
   }
-  __threadfence();
   __syncthreads();
   return *reinterpret_cast<volatile int*>(abort_sh) == 0;
 }
@@ -490,107 +317,176 @@ struct FusedArgs {
   int tiles_k, ntiles;
   int do_amax;                  // phase 1 runs (dynamic scale without RMSNorm)
   uint32_t* partials;           // [gridDim.x] written by phase 1
-  unsigned long long* flags;    // [2 * gridDim.x] barrier flags
+  unsigned long long* flags;    // barrier words: go words at [0] and [16], arrivals at [32 ..)
   unsigned long long epoch;     // this call's barrier epochs: epoch and epoch + 1
   uint64_t wait_ns;
   int mpad;                     // rows rounded up to 128 (scale padding rows)
 };
 
+// Shared-memory address of 16-byte chunk j (0..7) of tile row `row` in half h (channels
+// 64h .. 64h+63): each half is 128 rows x 128 bytes with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t qtile_chunk(uint32_t base, int h, int row, int j) {
+  return base + h * (128 * 128) + row * 128 + ((j ^ (row & 7)) << 4);
+}
+
+// Outlier list of one column tile: entries (j << 7) | (channel - k0) for the index-list
+// positions j whose channel falls in the tile, in increasing j.
+constexpr int kOCap = 256;  // entries per tile (128 distinct channels at most)
+struct OutlierList {
+  int n;
+  uint32_t e[kOCap];
+};
+
+// Codes of one resident tile, by one coding warp: lane l takes row 8w + l%8 and blocks l/8 and
+// 4 + l/8 of it (eight rows per 16-byte read hit eight distinct swizzled bank groups, and each
+// code store is 32 contiguous bytes in each of eight rows). Both blocks are loaded first and
+// coded side by side, and the lane writes its codes and scale bytes. Then the warp stashes the
+// outlier channels of its eight rows: lane l takes row l%8 and outlier entry l/8 (four entries
+// per pass), fetching the decode scale and code word of that element from the lane that coded
+// it by warp shuffles, and writes x (weights) or x minus its dequantized value (activations) to
+// column j of the stash. Nothing here waits for another warp.
+//   sf_lane: this lane's constant part of the scale offset, (mm%32)*16 + (mm/32)*4 + l/8
 template <bool RMS>
-__device__ __forceinline__ void code_tile(const QuantArgs& a, const uint8_t* tile, uint32_t tbase, int tm, int tk,
-                                          float s, float rcp_s, float rcp6, uint32_t* sf_tile, uint32_t* omask,
-                                          int16_t* ocol) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+__device__ __forceinline__ void code_rows(const QuantArgs& a, uint32_t tbase, int tm, int tk, float s, float rcp_s,
+                                          float rcp6, const OutlierList& ol, int sf_lane) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mm = warp * 8 + (lane & 7), bq = lane >> 3;
   const int m0 = tm * 128, k0 = tk * 128;
-  const int b = lane & 7, rsub = lane >> 3;
-  const int kcol = k0 + 16 * b;
-  const bool colok = kcol < a.K;
-  const uint32_t obits = (omask[b >> 1] >> ((b & 1) * 16)) & 0xFFFFu;
-  const int64_t cpitch = a.kpad >> 1;
-  uint8_t* sfb = reinterpret_cast<uint8_t*>(sf_tile);
-  float g[16];
-  if (RMS) {
-    uint4 g0 = make_uint4(0, 0, 0, 0), g1 = g0;
-    if (colok) {
-      g0 = ld_nc_v4(a.gain + kcol);
-      g1 = ld_nc_v4(a.gain + kcol + 8);
-    }
-    const uint32_t gs[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+  const int m = m0 + mm;
+  const bool rowok = m < a.M;
+  double inv = 0.0;
+  if (RMS) inv = rowok ? a.inv_rms[m] : 0.0;
+  uint32_t ws[2][8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) g[i] = (i & 1) ? bf16_hi(gs[i >> 1]) : bf16_lo(gs[i >> 1]);
+  for (int h = 0; h < 2; ++h) {
+    const uint4 w0 = lds_v4(qtile_chunk(tbase, h, mm, 2 * bq));
+    const uint4 w1 = lds_v4(qtile_chunk(tbase, h, mm, 2 * bq + 1));
+    ws[h][0] = w0.x, ws[h][1] = w0.y, ws[h][2] = w0.z, ws[h][3] = w0.w;
+    ws[h][4] = w1.x, ws[h][5] = w1.y, ws[h][6] = w1.z, ws[h][7] = w1.w;
   }
-  // 16 warps x 4 rows per step = 64 rows; two steps cover the 128-row tile
-#pragma unroll 1
-  for (int rg = 0; rg < 2; ++rg) {
-    const int mm = rg * 64 + warp * 4 + rsub;
-    const int m = m0 + mm;
-    const uint4 w0 = lds_v4(qtile_chunk(tbase, mm, 2 * b));
-    const uint4 w1 = lds_v4(qtile_chunk(tbase, mm, 2 * b + 1));
-    const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-    uint64_t p[8];
-    float amax;
-    double inv = 0.0;
+  float v[2][16];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int kcol = k0 + 16 * (4 * h + bq);
     if (RMS) {
-      inv = (m < a.M) ? a.inv_rms[m] : 0.0;
-      float mx = 0.0f;
+      uint4 g0 = make_uint4(0, 0, 0, 0), g1 = g0;
+      if (kcol < a.K) {
+        g0 = ld_nc_v4(a.gain + kcol);
+        g1 = ld_nc_v4(a.gain + kcol + 8);
+      }
+      const uint32_t gs[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const float v0 = rms_apply(bf16_lo(ws[j]), inv, g[2 * j]);
-        const float v1 = rms_apply(bf16_hi(ws[j]), inv, g[2 * j + 1]);
-        mx = fmaxf(mx, fmaxf(fabsf(v0), fabsf(v1)));
-        p[j] = f2_pack(v0, v1);
+        v[h][2 * j] = rms_apply(bf16_lo(ws[h][j]), inv, bf16_lo(gs[j]));
+        v[h][2 * j + 1] = rms_apply(bf16_hi(ws[h][j]), inv, bf16_hi(gs[j]));
       }
-      amax = mx;
     } else {
-      uint32_t am2 = 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        am2 = __vmaxu2(am2, ws[j] & 0x7FFF7FFFu);
-        p[j] = f2_pack(bf16_lo(ws[j]), bf16_hi(ws[j]));
-      }
-      amax = __uint_as_float(max(am2 & 0xFFFFu, am2 >> 16) << 16);
-    }
-    float d;
-    const uint32_t sfv = block_scale(amax, s, rcp_s, rcp6, &d);
-    const uint2 codes = (d == 0.0f) ? make_uint2(0u, 0u) : encode16(p, d);
-    if (m < a.M && colok) {
-      *reinterpret_cast<uint2*>(a.codes + static_cast<int64_t>(m) * cpitch + (kcol >> 1)) = codes;
-      sfb[(b >> 2) * 512 + (mm & 31) * 16 + (mm >> 5) * 4 + (b & 3)] = static_cast<uint8_t>(sfv);
-      uint32_t ob = obits;
-      while (ob) {
-        const int e = __ffs(ob) - 1;
-        ob &= ob - 1;
-        const uint32_t hv =
-            *reinterpret_cast<const uint16_t*>(tile + (qtile_chunk(tbase, mm, 2 * b + (e >> 3)) - tbase) + 2 * (e & 7));
-        float v = __uint_as_float(hv << 16);
-        if (RMS) v = rms_apply(v, inv, __bfloat162float(a.gain[kcol + e]));
-        const uint32_t c = ((e < 8 ? codes.x : codes.y) >> (4 * (e & 7))) & 15u;
-        const float deq = __fmul_rn(e2m1_value(c), d);
-        a.stash[static_cast<int64_t>(m) * a.r + ocol[16 * b + e]] = a.dup ? v : __fsub_rn(v, deq);
+        v[h][2 * j] = bf16_lo(ws[h][j]);
+        v[h][2 * j + 1] = bf16_hi(ws[h][j]);
       }
     }
+  }
+  float d[2];
+  uint32_t sfv[2];
+  uint2 codes[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const float a0 = fmax3_abs(v[h][0], v[h][1], v[h][2]), a1 = fmax3_abs(v[h][3], v[h][4], v[h][5]),
+                a2 = fmax3_abs(v[h][6], v[h][7], v[h][8]), a3 = fmax3_abs(v[h][9], v[h][10], v[h][11]),
+                a4 = fmax3_abs(v[h][12], v[h][13], v[h][14]);
+    sfv[h] = block_scale(fmaxf(fmax3(a0, a1, a2), fmax3(a3, a4, fabsf(v[h][15]))), s, rcp_s, rcp6, &d[h]);
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint64_t p[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) p[j] = f2_pack(v[h][2 * j], v[h][2 * j + 1]);
+    codes[h] = (d[h] == 0.0f) ? make_uint2(0u, 0u) : encode16(p, d[h]);
+  }
+  uint8_t* crow = a.codes + static_cast<int64_t>(rowok ? m : 0) * (a.kpad >> 1) + (k0 >> 1);
+  uint8_t* sft = a.sf + (static_cast<int64_t>(tm) * a.katoms + (k0 >> 6)) * 512 + sf_lane;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    if (k0 + 16 * (4 * h + bq) >= a.K) continue;
+    if (rowok) *reinterpret_cast<uint2*>(crow + 8 * (4 * h + bq)) = codes[h];
+    // padding rows (up to the next multiple of 128) carry zero scales
+    sft[h * 512] = rowok ? static_cast<uint8_t>(sfv[h]) : 0;
+  }
+  // outlier channels of the warp's eight rows, four entries per pass (the lane keeps its row)
+  for (int base = 0; base < ol.n; base += 4) {
+    const int o = base + (lane >> 3);
+    const bool act = o < ol.n && rowok;
+    const uint32_t ent = (o < ol.n) ? ol.e[o] : 0u;
+    const int col = static_cast<int>(ent & 127u), j = static_cast<int>(ent >> 7);
+    const int blk = col >> 4, e = col & 15;
+    const int src = (lane & 7) + 8 * (blk & 3);  // the lane that coded (this row, block blk)
+    const float dd0 = __shfl_sync(0xFFFFFFFFu, d[0], src), dd1 = __shfl_sync(0xFFFFFFFFu, d[1], src);
+    const uint32_t c0x = __shfl_sync(0xFFFFFFFFu, codes[0].x, src), c0y = __shfl_sync(0xFFFFFFFFu, codes[0].y, src);
+    const uint32_t c1x = __shfl_sync(0xFFFFFFFFu, codes[1].x, src), c1y = __shfl_sync(0xFFFFFFFFu, codes[1].y, src);
+    if (!act) continue;
+    uint16_t hv;
+    asm volatile("ld.shared.u16 %0, [%1];"
+                 : "=h"(hv)
+                 : "r"(qtile_chunk(tbase, blk >> 2, mm, (col & 63) >> 3) + 2 * (col & 7)));
+    float x = __uint_as_float(static_cast<uint32_t>(hv) << 16);
+    if (RMS) x = rms_apply(x, inv, __bfloat162float(a.gain[k0 + col]));
+    float res = x;
+    if (!a.dup) {
+      const uint32_t cw = (blk >> 2) ? ((e < 8) ? c1x : c1y) : ((e < 8) ? c0x : c0y);
+      const uint32_t c = (cw >> (4 * (e & 7))) & 15u;
+      res = __fsub_rn(x, __fmul_rn(e2m1_value(c), (blk >> 2) ? dd1 : dd0));
+    }
+    a.stash[static_cast<int64_t>(j) * a.M + m] = res;
   }
 }
 
-// The appended residual blocks (from the stash) and zero padding up to K_pad of one row.
-__device__ __forceinline__ void tail_row(const QuantArgs& a, int m, float s, float rcp_s, float rcp6, int lane) {
+// The outlier list of column tile k0 .. k0+127, by one warp (ballot compaction).
+__device__ __forceinline__ void build_olist(const QuantArgs& a, const int32_t* idx_sh, int k0, OutlierList& ol,
+                                            int lane) {
+  int n = 0;
+  for (int base = 0; base < a.r; base += 32) {
+    const int j = base + lane;
+    const int c = (j < a.r) ? (j < kIdxSmem ? idx_sh[j] : __ldg(a.idx + j)) : -1;
+    const bool hit = j < a.r && c < a.K && static_cast<unsigned>(c - k0) < 128u;
+    const uint32_t mask = __ballot_sync(0xFFFFFFFFu, hit);
+    const int pos = n + __popc(mask & ((1u << lane) - 1u));
+    if (hit && pos < kOCap) ol.e[pos] = (static_cast<uint32_t>(j) << 7) | static_cast<uint32_t>(c - k0);
+    n += __popc(mask);
+  }
+  if (n > kOCap) {
+    if (lane == 0) set_status(kStatusInvalidArg);  // more entries than distinct channels
+    n = kOCap;
+  }
+  if (lane == 0) ol.n = n;
+  __syncwarp();
+}
+
+// The appended residual blocks (from the stash) and zero padding up to K_pad: one (row, block)
+// per thread, rows fastest.
+__device__ __forceinline__ void tail_items(const QuantArgs& a, int mpad, float s, float rcp_s, float rcp6) {
   const int nres = a.r >> 4;
   const int ntail = (a.kpad - a.K) >> 4;
   const int64_t cpitch = a.kpad >> 1;
-  for (int b = lane; b < ntail; b += 32) {
+  const int64_t items = static_cast<int64_t>(mpad) * ntail;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t it = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it < items; it += stride) {
+    const int b = static_cast<int>(it / mpad), m = static_cast<int>(it - static_cast<int64_t>(b) * mpad);
     uint32_t sfv = 0;
     uint2 codes = make_uint2(0u, 0u);
     if (m < a.M && b < nres) {
-      const float4* src = reinterpret_cast<const float4*>(a.stash + static_cast<int64_t>(m) * a.r + 16 * b);
-      uint64_t p[8];
-      float am = 0.0f;
+      const float* src = a.stash + static_cast<int64_t>(16 * b) * a.M + m;
+      float v[16];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 q = src[i];
-        p[2 * i] = f2_pack(q.x, q.y);
-        p[2 * i + 1] = f2_pack(q.z, q.w);
-        am = fmaxf(am, fmaxf(fmaxf(fabsf(q.x), fabsf(q.y)), fmaxf(fabsf(q.z), fabsf(q.w))));
-      }
+      for (int i = 0; i < 16; ++i) v[i] = __ldcg(src + static_cast<int64_t>(i) * a.M);
+      uint64_t p[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) p[j] = f2_pack(v[2 * j], v[2 * j + 1]);
+      const float a0 = fmax3_abs(v[0], v[1], v[2]), a1 = fmax3_abs(v[3], v[4], v[5]),
+                  a2 = fmax3_abs(v[6], v[7], v[8]), a3 = fmax3_abs(v[9], v[10], v[11]),
+                  a4 = fmax3_abs(v[12], v[13], v[14]);
+      const float am = fmaxf(fmax3(a0, a1, a2), fmax3(a3, a4, fabsf(v[15])));
       float d;
       sfv = block_scale(am, s, rcp_s, rcp6, &d);
       if (d != 0.0f) codes = encode16(p, d);
@@ -605,76 +501,108 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_quant_fused(const __grid_c
                                                                   QuantArgs a, FusedArgs f) {
   extern __shared__ uint8_t fsmem_raw[];
   uint8_t* qs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fsmem_raw) + 1023) & ~uintptr_t(1023));
-  uint32_t* sf_tile = reinterpret_cast<uint32_t*>(qs + kFusedBufs * kQTileBytes);
-  __shared__ uint64_t bar[kFusedBufs];
-  __shared__ uint32_t omask[4];
-  __shared__ int16_t ocol[128];
+  __shared__ uint64_t full[kFusedBufs], empty[kFusedBufs];
+  __shared__ int32_t idx_sh[kIdxSmem];
+  __shared__ OutlierList olist[kFusedBufs];  // outlier list of the tile in each ring buffer
   __shared__ int abort_sh;
-  __shared__ int issued_sh;  // slots whose loads thread 0 has issued
   __shared__ float s_sh;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool producer = warp == kCodeWarps;
   const int G = gridDim.x;
   const int n_c = (f.ntiles > static_cast<int>(blockIdx.x)) ? (f.ntiles - blockIdx.x + G - 1) / G : 0;
   const uint32_t xbase = smem_u32(qs);
-  auto tile_of = [&](int i) { return static_cast<int>(blockIdx.x) + i * G; };  // CTA-local index -> tile
-  auto issue = [&](int slot, int i) {
-    const int t = tile_of(i);
-    const int tm = t / f.tiles_k, tk = t - (t / f.tiles_k) * f.tiles_k;
+  // CTA-local tile i is tile blockIdx.x + i * G. Phase 1 streams i = 0 .. n_c-1 through slots
+  // 0 .. n_c-1 and leaves the last `resident` of them in the ring; phase 2 codes those first,
+  // then the others, which come through the ring again. Slot sl uses buffer sl % kFusedBufs.
+  const int resident = f.do_amax ? min(n_c, kFusedBufs) : 0;
+  const int first_slot = f.do_amax ? n_c - resident : 0;  // slot of processing position q = 0
+  auto tile_at = [&](int q) {
+    const int i = f.do_amax ? (q < resident ? n_c - resident + q : q - resident) : q;
+    return static_cast<int>(blockIdx.x) + i * G;
+  };
+  int issued = 0;  // producer lane 0: slots issued so far
+  auto issue = [&](int slot, int t) {
+    const int tm = t / f.tiles_k, tk = t - tm * f.tiles_k;
     const int buf = slot % kFusedBufs;
-    mbar_arrive_expect_tx(&bar[buf], kQTileBytes);
+    mbar_arrive_expect_tx(&full[buf], kQTileBytes);
     uint8_t* dst = qs + buf * kQTileBytes;
-    tma_load_2d(dst, &tmX, &bar[buf], tk * 128, tm * 128);
-    tma_load_2d(dst + 128 * 128, &tmX, &bar[buf], tk * 128 + 64, tm * 128);
-    issued_sh = slot + 1;
+    tma_load_2d(dst, &tmX, &full[buf], tk * 128, tm * 128);
+    tma_load_2d(dst + 128 * 128, &tmX, &full[buf], tk * 128 + 64, tm * 128);
+    issued = slot + 1;
   };
-  auto wait_slot = [&](int slot) -> bool {
-    if (!mbar_wait(&bar[slot % kFusedBufs], static_cast<uint32_t>((slot / kFusedBufs) & 1), f.wait_ns, &abort_sh))
-      abort_sh = 1;
-    __syncthreads();
-    return abort_sh == 0;
+  // producer: before reusing a buffer, wait until the coding warps released its previous slot
+  // (sleeping between polls, so the wait leaves the issue slots to the coding warps)
+  auto wait_free = [&](int slot) -> bool {
+    if (slot < kFusedBufs) return true;
+    return mbar_wait(&empty[slot % kFusedBufs], static_cast<uint32_t>((slot / kFusedBufs - 1) & 1), f.wait_ns,
+                     &abort_sh, 128);
   };
-  // after an abort: let every load still in flight land (bounded) before the CTA exits
-  auto teardown = [&](int from_slot) {
-    if (tid == 0) {
-      const uint64_t t0 = globaltimer_ns();
-      for (int sl = from_slot; sl < issued_sh; ++sl)
-        while (!mbar_test(&bar[sl % kFusedBufs], static_cast<uint32_t>((sl / kFusedBufs) & 1)) &&
-               globaltimer_ns() - t0 < f.wait_ns) {
-        }
+  // producer lane 0 after an abort: the last load issued into each buffer lands (bounded)
+  auto drain = [&]() {
+    const uint64_t t0 = globaltimer_ns();
+    for (int b = 0; b < kFusedBufs; ++b) {
+      int sl = issued - 1 - ((issued - 1 - b) % kFusedBufs + kFusedBufs) % kFusedBufs;
+      if (sl < 0) continue;
+      while (!mbar_test(&full[b], static_cast<uint32_t>((sl / kFusedBufs) & 1)) && globaltimer_ns() - t0 < f.wait_ns) {
+      }
     }
   };
-  if (tid == 0) {
-    for (int i = 0; i < kFusedBufs; ++i) mbar_init(&bar[i], 1);
+  auto release = [&](int slot) {  // coding warp done with the slot's buffer and outlier list
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[slot % kFusedBufs]);
+  };
+  // A full barrier completes on the tile's bytes plus two producer arrivals: one with the
+  // byte count when the loads are issued, one when the tile's outlier list is written.
+  if (producer && lane == 0) {
+    for (int i = 0; i < kFusedBufs; ++i) {
+      mbar_init(&full[i], 2);
+      mbar_init(&empty[i], kCodeWarps);
+    }
     abort_sh = 0;
-    issued_sh = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmX);
-    for (int i = 0; i < min(n_c, kFusedBufs); ++i) issue(i, i);
+    // the first kFusedBufs slots hold tiles 0 .. kFusedBufs-1 in either phase order
+    for (int sl = 0; sl < min(n_c, kFusedBufs); ++sl) issue(sl, static_cast<int>(blockIdx.x) + sl * G);
   }
+  for (int j = tid; j < min(a.r, kIdxSmem); j += kFusedThreads) idx_sh[j] = a.idx[j];
+  if (blockIdx.x == 0)
+    for (int j = tid; j < a.r; j += kFusedThreads)
+      if (static_cast<unsigned>(a.idx[j]) >= static_cast<unsigned>(a.K)) set_status(kStatusInvalidArg);
   __syncthreads();
-  int slot = 0;     // next slot to consume
-  int resident = 0;  // tiles left in the ring by phase 1 (CTA-local indices n_c-resident .. n_c-1)
   if (f.do_amax) {
     // ------------------------------------------------------------------ phase 1: max |x|
     uint32_t mx = 0;
-    for (int i = 0; i < n_c; ++i, ++slot) {
-      if (!wait_slot(slot)) {
-        teardown(slot);
-        return;
+    if (producer) {
+      if (lane == 0) {
+        for (int sl = 0; sl < n_c; ++sl) {
+          if (sl >= kFusedBufs) {
+            if (!wait_free(sl)) break;
+            issue(sl, static_cast<int>(blockIdx.x) + sl * G);
+          }
+          mbar_arrive(&full[sl % kFusedBufs]);  // phase 1 reads no outlier list
+        }
       }
-      const uint32_t tb = xbase + (slot % kFusedBufs) * kQTileBytes;
-      // 512 threads x 4 chunks of 16 bytes = the 32 KB tile
+      __syncwarp();
+      // outlier lists of the tiles that stay resident (their buffers hold no list in phase 1;
+      // the grid barrier below publishes them)
+      for (int sl = first_slot; sl < n_c; ++sl)
+        build_olist(a, idx_sh, (tile_at(sl - first_slot) % f.tiles_k) * 128, olist[sl % kFusedBufs], lane);
+    } else {
+      for (int sl = 0; sl < n_c; ++sl) {
+        const int buf = sl % kFusedBufs;
+        if (!mbar_wait(&full[buf], static_cast<uint32_t>((sl / kFusedBufs) & 1), f.wait_ns, &abort_sh)) break;
+        const uint32_t tb = xbase + buf * kQTileBytes;
+        // 512 threads x 4 chunks of 16 bytes = the 32 KB tile
 #pragma unroll
-      for (int j = 0; j < 4; ++j) mx = absmax_bf16x2(mx, lds_v4(tb + (tid + j * kFusedThreads) * 16));
-      __syncthreads();
-      if (tid == 0 && i + kFusedBufs < n_c) {
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        issue(slot + kFusedBufs, i + kFusedBufs);
+        for (int j = 0; j < 4; ++j) mx = absmax_bf16x2(mx, lds_v4(tb + (tid + j * kCodeWarps * 32) * 16));
+        if (sl < first_slot) release(sl);
       }
     }
     cta_max_to(max(mx & 0xFFFFu, mx >> 16) << 16, &f.partials[blockIdx.x]);
-    resident = min(n_c, kFusedBufs);
-    if (!grid_barrier(f.flags, G, f.epoch, f.wait_ns, &abort_sh)) return;
+    if (!grid_barrier(f.flags + 32, f.flags, G, f.epoch, f.wait_ns, &abort_sh)) {
+      if (producer && lane == 0) drain();
+      return;
+    }
   }
   // ---------------------------------------------------------------------- phase 2: code tiles
   {
@@ -690,92 +618,44 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_quant_fused(const __grid_c
   const float s = s_sh;
   if (blockIdx.x == 0 && tid == 0) *a.scale_out = s;
   const float rcp_s = __frcp_rn(s), rcp6 = __frcp_rn(6.0f);
-  // processing order: the resident tiles (slots n_c-resident .. n_c-1), then the rest
-  const int first_slot = f.do_amax ? n_c - resident : 0;
-  const int nproc = n_c;
-  for (int q = 0; q < nproc; ++q) {
-    const int cur = first_slot + q;  // slot of this tile
-    const int i = f.do_amax ? (q < resident ? n_c - resident + q : q - resident) : q;
-    const int t = tile_of(i);
-    const int tm = t / f.tiles_k, tk = t - tm * f.tiles_k;
-    const int k0 = tk * 128;
-    __syncthreads();
-    for (int j = tid; j < 256; j += kFusedThreads) sf_tile[j] = 0;
-    if (tid < 4) omask[tid] = 0;
-    __syncthreads();
-    for (int j = tid; j < a.r; j += kFusedThreads) {
-      const int c = a.idx[j];
-      if (c >= k0 && c < k0 + 128) {
-        ocol[c - k0] = static_cast<int16_t>(j);
-        atomicOr(&omask[(c - k0) >> 5], 1u << ((c - k0) & 31));
+  if (producer) {
+    for (int q = resident; q < n_c; ++q) {
+      const int sl = first_slot + q, buf = sl % kFusedBufs;
+      const int t = tile_at(q);
+      bool ok = true;
+      if (lane == 0 && sl >= kFusedBufs) {  // the first kFusedBufs slots were issued at the start
+        ok = wait_free(sl);
+        if (ok) issue(sl, t);
       }
+      if (!__shfl_sync(0xFFFFFFFFu, static_cast<int>(ok), 0)) break;
+      build_olist(a, idx_sh, (t % f.tiles_k) * 128, olist[buf], lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full[buf]);
     }
-    const bool loaded = f.do_amax && q < resident;  // already waited for in phase 1
-    if (!loaded) {
-      if (!wait_slot(cur)) {
-        teardown(cur);
-        return;
-      }
-    } else {
-      __syncthreads();
+  } else {
+    const int mm = warp * 8 + (lane & 7);
+    const int sf_lane = (mm & 31) * 16 + (mm >> 5) * 4 + (lane >> 3);
+    for (int q = 0; q < n_c; ++q) {
+      const int sl = first_slot + q, buf = sl % kFusedBufs;
+      const int t = tile_at(q);
+      const int tm = t / f.tiles_k, tk = t - tm * f.tiles_k;
+      // resident tiles were waited for in phase 1
+      if (q >= resident &&
+          !mbar_wait(&full[buf], static_cast<uint32_t>((sl / kFusedBufs) & 1), f.wait_ns, &abort_sh))
+        break;
+      code_rows<RMS>(a, xbase + buf * kQTileBytes, tm, tk, s, rcp_s, rcp6, olist[buf], sf_lane);
+      release(sl);
     }
-    const int buf = cur % kFusedBufs;
-    code_tile<RMS>(a, qs + buf * kQTileBytes, xbase + buf * kQTileBytes, tm, tk, s, rcp_s, rcp6, sf_tile, omask,
-                   ocol);
-    __syncthreads();
-    // the next load into this buffer: the tile kFusedBufs slots later, if any
-    const int next = q + kFusedBufs;
-    if (tid == 0 && next < nproc) {
-      const int inext = f.do_amax ? (next < resident ? -1 : next - resident) : next;
-      if (inext >= 0) {
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        issue(cur + kFusedBufs, inext);
-      }
-    }
-    const int natoms = min(2, (a.K - k0 + 63) >> 6);
-    uint4* dst = reinterpret_cast<uint4*>(a.sf + (static_cast<int64_t>(tm) * a.katoms + (k0 >> 6)) * 512);
-    const uint4* src = reinterpret_cast<const uint4*>(sf_tile);
-    for (int j = tid; j < natoms * 32; j += kFusedThreads) dst[j] = src[j];
+  }
+  __syncthreads();  // both roles are done with the ring
+  if (abort_sh) {
+    if (producer && lane == 0) drain();
+    return;
   }
   if (a.kpad == a.K) return;
   // ---------------------------------------------------------------------- phase 3: tail
-  if (!grid_barrier(f.flags + G, G, f.epoch + 1, f.wait_ns, &abort_sh)) return;
-  const int warp = tid >> 5, lane = tid & 31;
-  for (int m = blockIdx.x * (kFusedThreads / 32) + warp; m < f.mpad; m += G * (kFusedThreads / 32))
-    tail_row(a, m, s, rcp_s, rcp6, lane);
-}
-
-// One warp per row (rows up to the 128-padded count): appended residual blocks and padding.
-__global__ void __launch_bounds__(256) k_quant_tail(QuantArgs a, int mpad) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m = blockIdx.x * 8 + warp;
-  if (m >= mpad) return;
-  const float s = (a.static_scale) ? *a.static_scale : *a.scale_out;
-  const float rcp_s = __frcp_rn(s), rcp6 = __frcp_rn(6.0f);
-  const int nres = a.r >> 4;
-  const int ntail = (a.kpad - a.K) >> 4;
-  const int64_t cpitch = a.kpad >> 1;
-  for (int b = lane; b < ntail; b += 32) {
-    uint32_t sfv = 0;
-    uint2 codes = make_uint2(0u, 0u);
-    if (m < a.M && b < nres) {
-      const float4* src = reinterpret_cast<const float4*>(a.stash + static_cast<int64_t>(m) * a.r + 16 * b);
-      uint64_t p[8];
-      float am = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 q = src[i];
-        p[2 * i] = f2_pack(q.x, q.y);
-        p[2 * i + 1] = f2_pack(q.z, q.w);
-        am = fmaxf(am, fmaxf(fmaxf(fabsf(q.x), fabsf(q.y)), fmaxf(fabsf(q.z), fabsf(q.w))));
-      }
-      float d;
-      sfv = block_scale(am, s, rcp_s, rcp6, &d);
-      if (d != 0.0f) codes = encode16(p, d);
-    }
-    if (m < a.M) *reinterpret_cast<uint2*>(a.codes + static_cast<int64_t>(m) * cpitch + ((a.K + 16 * b) >> 1)) = codes;
-    a.sf[sf_offset(m, (a.K >> 4) + b, a.katoms)] = static_cast<uint8_t>(sfv);
-  }
+  if (!grid_barrier(f.flags + 32 + G, f.flags + 16, G, f.epoch + 1, f.wait_ns, &abort_sh)) return;
+  tail_items(a, f.mpad, s, rcp_s, rcp6);
 }
 
 }  // namespace arc
