@@ -8,21 +8,33 @@
 //   FP4 = false: BF16 GEMM (tcgen05.mma kind::f16), the reference-precision switch of RAMP
 //                (section 4.1: the recurrent steps after the switch run in BF16).
 //
-// CTA = 10 warps, one CTA per SM, persistent over 128 x 256 output tiles (grouped raster):
-//   warp 0      TMA producer: A tile 128 rows x 128 bytes and B tile 256 rows x 128 bytes per
-//               stage (128-byte swizzle), plus the stage's scale atoms as 1-D bulk copies (A:
-//               up to 4 atoms of its 128-row block, B: up to 4 atoms of each of its two
-//               128-row blocks); no multicast.
-//   warp 1      TMEM allocation and MMA issue (one thread): per stage, tcgen05.cp of the scale
-//               atoms into TMEM (32x128b, replicated to the four lane quarters), then 4 MMAs of
-//               K = 64 (fp4) / 16 (bf16), committed to the stage's "empty" barrier.
-//   warps 2..9  epilogue: tcgen05.ld of the fp32 accumulator (warp w owns TMEM lanes
-//               32*(w%4)..+31 = tile rows, and one 128-column half), scale by alpha, optional
-//               residual add, bf16 stores.
-// TMEM: fp32 accumulator 128 lanes x 256 columns (two of them for bf16; fp4 keeps one and puts
-// the scale factors in columns 256..303). Every wait is bounded (wait_ns); a wait that runs out
-// raises the CTA's abort flag and the device status word, and the CTA drains what it issued
-// and frees its tensor memory before it returns.
+// CTA = 15 warps, one CTA per SM, persistent over 128 x 256 output tiles (grouped raster):
+//   warp 0       TMA producer: per stage an A tile of 128 rows x 128 bytes and a B tile of 256
+//                rows x 128 bytes (128-byte swizzle), plus the stage's scale atoms as 1-D bulk
+//                copies (A: up to 4 atoms of its 128-row block; B: up to 4 atoms of each of its
+//                two 128-row blocks); no multicast.
+//   warps 1, 2   MMA issue (one thread each), alternating pipeline stages: warp 1 takes the
+//                even stages, warp 2 the odd ones. A single issuing thread that waits for every
+//                stage leaves the tensor pipe idle for a while after each wait; two issuers
+//                cover each other's waits. A shared issue ticket (release/acquire, bracketed
+//                with tcgen05 fences) keeps the stages entering the tensor pipe in order, so the
+//                fp32 accumulation order is fixed and results are reproducible bit for bit.
+//                Warp 1 also owns the TMEM allocation.
+//   warps 3..6   (FP4) scale writers, one per TMEM lane quarter: they read the stage's scale
+//                bytes from shared memory and store them into the stage's set of TMEM scale
+//                columns with tcgen05.st, in the cell order the block-scaled MMA reads
+//                (A: row m at lane m, column base + m/32; B: column n at lane 32q + n%32 of
+//                every quarter q, column base + n/32). Register stores keep the tensor pipe free
+//                for MMAs; tcgen05.cp of the same bytes costs the pipe ~70 cycles per copy.
+//   warps 7..14  epilogue: tcgen05.ld of the fp32 accumulator (warp w owns TMEM lane quarter
+//                w%4 = tile rows 32*(w%4)..+31, and one 128-column half), scale by alpha,
+//                optional residual add, bf16 stores.
+// TMEM (512 columns): fp32 accumulator 128 lanes x 256 columns (two of them for bf16); fp4
+// keeps one and uses columns 256..511 as four 64-column scale sets, one per pipeline stage
+// (B scales at +0..31, 8 columns per K=64 step; A scales at +32 + 4k + quarter).
+// Every wait is bounded (wait_ns); a wait that runs out raises the CTA's abort flag and the
+// device status word, and the CTA drains what it issued and frees its tensor memory before it
+// returns.
 #pragma once
 
 #include "arc_device.cuh"
@@ -40,7 +52,7 @@ struct GemmTraits<true> {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr uint32_t IDESC = idesc_nvf4(BM, BN);
   static constexpr int TMEM_COLS = 512;
-  static constexpr int SFA_COL = 256, SFB_COL = 272;
+  static constexpr int SF_COL0 = 256, SF_SET_COLS = 64;
 };
 
 template <>
@@ -51,7 +63,7 @@ struct GemmTraits<false> {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t IDESC = idesc_bf16(BM, BN);
   static constexpr int TMEM_COLS = 512;
-  static constexpr int SFA_COL = 0, SFB_COL = 0;
+  static constexpr int SF_COL0 = 0, SF_SET_COLS = 0;
 };
 
 template <bool FP4>
@@ -98,7 +110,29 @@ __device__ __forceinline__ void mbar_wait_teardown(uint64_t* bar, uint32_t parit
   }
 }
 
-constexpr int kGemmThreads = 320;  // producer warp, MMA warp, 8 epilogue warps
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint4 lds_u32x4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// CTA-scope release store / acquire load of a shared-memory flag.
+__device__ __forceinline__ void st_release_cta(int* p, int v) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_cta(const int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+
+constexpr int kGemmThreads = 480;  // producer, 2 MMA issuers, 4 scale writers, 8 epilogue warps
+constexpr int kGemmEpiWarp0 = 7;
 
 template <bool FP4, bool ADD>
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -108,24 +142,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + T::STAGES * T::STAGE_BYTES);
   uint64_t* empty = full + T::STAGES;
-  uint64_t* acc_full = empty + T::STAGES;
+  uint64_t* ready = empty + T::STAGES;  // fp4: the stage's scales are in TMEM
+  uint64_t* acc_full = ready + T::STAGES;
   uint64_t* acc_empty = acc_full + 2;
-  uint64_t* drain = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain = acc_empty + 2;  // one per MMA warp
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* issued = reinterpret_cast<int*>(tmem_slot + 2);  // pipeline stages whose MMAs are issued
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < T::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&ready[s], 4);
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 8);
+      mbar_init(&acc_full[a], 2);   // one commit from each MMA warp per tile
+      mbar_init(&acc_empty[a], 8);  // one arrival from each epilogue warp
     }
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
+    st_release_cta(issued, 0);
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
@@ -193,71 +232,129 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if ((armed >> s) & 1u) mbar_wait_teardown(&full[s], (armed_par >> s) & 1u, g.wait_ns);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 2) {
     if (lane == 0) {
-      // ------------------------------------------------------------------ MMA issuer
-      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      // ------------------------------------------------------------------ MMA issue
+      const int me = warp - 1;
+      uint32_t acc = 0, acc_phase = 0;
+      int seq = 0;  // pipeline stage counter, the same sequence the producer walks
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        // the accumulator must have been drained by the epilogue (also keeps this warp's
+        // acc_full commits one tile apart)
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, g.wait_ns, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + acc * T::BN;
-        for (int ks = 0; ks < g.kstages; ++ks) {
-          if (!mbar_wait(&full[stage], phase, g.wait_ns, abort_flag)) {
+        for (int ks = 0; ks < g.kstages; ++ks, ++seq) {
+          if ((seq & 1) != me) continue;
+          const int stage = seq % T::STAGES;
+          const uint32_t par = static_cast<uint32_t>((seq / T::STAGES) & 1);
+          if (!mbar_wait(FP4 ? &ready[stage] : &full[stage], par, g.wait_ns, abort_flag)) {
             ok = false;
             break;
+          }
+          // issue ticket: every earlier stage (the other warp's) is in the tensor pipe first, so
+          // the accumulation order, and with it the result, does not depend on timing
+          if (ld_acquire_cta(issued) != seq) {
+            const uint64_t t0 = globaltimer_ns();
+            while (ld_acquire_cta(issued) != seq) {
+              if (*abort_flag || globaltimer_ns() - t0 > g.wait_ns) {
+                *abort_flag = 1;
+                set_status(kStatusTimeout);
+                ok = false;
+                break;
+              }
+            }
+            if (!ok) break;
           }
           tc_fence_after();
           uint8_t* sA = smem + stage * T::STAGE_BYTES;
           uint8_t* sB = sA + T::A_BYTES;
           const int nk = FP4 ? min(4, g.ksteps - 4 * ks) : 4;
-          if (FP4) {
-            uint8_t* sSFA = sB + T::B_BYTES;
-            uint8_t* sSFB = sSFA + T::SFA_BYTES;
-            for (int k = 0; k < nk; ++k) {
-              tc_cp_sf_atom(tmem + T::SFA_COL + 4 * k, desc_sf_atom(smem_u32(sSFA + k * 512)));
-              tc_cp_sf_atom(tmem + T::SFB_COL + 8 * k, desc_sf_atom(smem_u32(sSFB + k * 512)));
-              tc_cp_sf_atom(tmem + T::SFB_COL + 8 * k + 4, desc_sf_atom(smem_u32(sSFB + 2048 + k * 512)));
-            }
-          }
           const uint64_t da = desc_kmajor_sw128(smem_u32(sA));
           const uint64_t db = desc_kmajor_sw128(smem_u32(sB));
+          const uint32_t sf = tmem + T::SF_COL0 + T::SF_SET_COLS * stage;
           for (int k = 0; k < nk; ++k) {
             const uint64_t off = static_cast<uint64_t>((k * 32) >> 4);
             const uint32_t accum = (ks > 0 || k > 0) ? 1u : 0u;
             if (FP4)
-              tc_mma_nvf4(d_tmem, da + off, db + off, T::IDESC, tmem + T::SFA_COL + 4 * k, tmem + T::SFB_COL + 8 * k,
-                          accum);
+              tc_mma_nvf4(d_tmem, da + off, db + off, T::IDESC, sf + 32 + 4 * k, sf + 8 * k, accum);
             else
               tc_mma_bf16(d_tmem, da + off, db + off, T::IDESC, accum);
           }
           tc_commit(&empty[stage]);
-          if (++stage == T::STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
+          tc_fence_before();
+          st_release_cta(issued, seq + 1);
         }
         if (!ok) break;
-        tc_commit(&acc_full[acc]);
+        tc_commit(&acc_full[acc]);  // every MMA warp, once per tile (acc_full counts two)
         if (++acc == T::ACC_STAGES) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
       // nothing issued may still be running when the tensor memory is released
-      tc_commit(drain);
-      mbar_wait_teardown(drain, 0, g.wait_ns);
+      tc_commit(&drain[me]);
+      mbar_wait_teardown(&drain[me], 0, g.wait_ns);
+    }
+  } else if (warp < kGemmEpiWarp0) {
+    if (FP4) {
+      // ------------------------------------------------------------------ scale writers
+      const int q = warp & 3;
+      const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        for (int ks = 0; ks < g.kstages; ++ks) {
+          const bool got = mbar_wait(&full[stage], phase, g.wait_ns, abort_flag);
+          if (!__all_sync(0xFFFFFFFFu, got)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int natoms = min(4, g.katoms - 4 * ks);
+          const uint32_t sSFA = smem_u32(smem + stage * T::STAGE_BYTES + T::A_BYTES + T::B_BYTES);
+          const uint32_t sSFB = sSFA + T::SFA_BYTES;
+          uint32_t v[32];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            uint4 b0 = make_uint4(0, 0, 0, 0), b1 = b0;
+            if (k < natoms) {
+              b0 = lds_u32x4(sSFB + k * 512 + lane * 16);
+              b1 = lds_u32x4(sSFB + 2048 + k * 512 + lane * 16);
+            }
+            v[8 * k + 0] = b0.x, v[8 * k + 1] = b0.y, v[8 * k + 2] = b0.z, v[8 * k + 3] = b0.w;
+            v[8 * k + 4] = b1.x, v[8 * k + 5] = b1.y, v[8 * k + 6] = b1.z, v[8 * k + 7] = b1.w;
+          }
+          const uint32_t set = lane_base + T::SF_COL0 + T::SF_SET_COLS * stage;
+          tmem_st_32x32b_x32(set, v);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t a = (k < natoms) ? lds_u32(sSFA + k * 512 + lane * 16 + 4 * q) : 0u;
+            tmem_st_32x32b_x1(set + 32 + 4 * k + q, a);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ready[stage]);
+          if (++stage == T::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
     }
   } else {
     // -------------------------------------------------------------------- epilogue
     // 8 warps: warp w reads TMEM lane quarter w%4 (tile rows 32*(w%4)..+31) and column half
-    // (w-2)/4 (128 columns). Without a residual add the warp pulls its whole 32 x 128 block out
-    // of TMEM in one burst and releases the accumulator before it converts and stores; with an
-    // add, the residual block is prefetched into registers and the accumulator is read and
+    // (w-7)/4 (128 columns). Without a residual add the warp converts its 32 x 128 block to
+    // bf16 chunk by chunk as it leaves TMEM, releases the accumulator, then stores; with an add,
+    // the residual block is prefetched into registers and the accumulator is read, combined and
     // stored 32 columns at a time.
     const int q = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int half = (warp - kGemmEpiWarp0) >> 2;
     const float alpha = FP4 ? __fmul_rn(*g.a_scale, *g.b_scale) : 1.0f;
+    const uint64_t alpha2 = f2_pack(alpha, alpha);
     constexpr int HB = T::BN / 2;  // columns per warp
     uint32_t acc = 0, acc_phase = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
@@ -282,43 +379,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       // every lane waits; the warp goes on only if all of them saw the accumulator (the TMEM
       // loads below are warp-collective, so the decision must be uniform)
-      const bool ready = mbar_wait(&acc_full[acc], acc_phase, g.wait_ns, abort_flag, 64);
-      if (!__all_sync(0xFFFFFFFFu, ready)) break;
+      const bool got = mbar_wait(&acc_full[acc], acc_phase, g.wait_ns, abort_flag, 64);
+      if (!__all_sync(0xFFFFFFFFu, got)) break;
       tc_fence_after();
       const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * T::BN + half * HB;
       if (!ADD) {
-        uint32_t r[HB / 32][32];
+        uint32_t pk[HB / 2];
 #pragma unroll
-        for (int c = 0; c < HB / 32; ++c) tmem_ld_32x32b_x32(tbase + c * 32, r[c]);
-        tmem_ld_wait();
+        for (int c = 0; c < HB / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tbase + c * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float a0, a1;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), alpha2), a0, a1);
+            pk[16 * c + e] = pack_bf16x2_rn(a0, a1);
+          }
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[acc]);
         if (row_ok) {
 #pragma unroll
-          for (int c = 0; c < HB / 32; ++c) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int col = col0 + c * 32 + 8 * j;
-              if (col < g.N) {
-                uint64_t f[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                  f[e] = f2_mul(f2_pack(__uint_as_float(r[c][8 * j + 2 * e]), __uint_as_float(r[c][8 * j + 2 * e + 1])),
-                                f2_pack(alpha, alpha));
-                uint4 o;
-                float a0, a1;
-                f2_unpack(f[0], a0, a1);
-                o.x = pack_bf16x2_rn(a0, a1);
-                f2_unpack(f[1], a0, a1);
-                o.y = pack_bf16x2_rn(a0, a1);
-                f2_unpack(f[2], a0, a1);
-                o.z = pack_bf16x2_rn(a0, a1);
-                f2_unpack(f[3], a0, a1);
-                o.w = pack_bf16x2_rn(a0, a1);
-                *reinterpret_cast<uint4*>(yrow + col) = o;
-              }
-            }
+          for (int j = 0; j < HB / 8; ++j) {
+            const int col = col0 + 8 * j;
+            if (col < g.N)
+              *reinterpret_cast<uint4*>(yrow + col) = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
           }
         }
       } else {
