@@ -24,7 +24,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -86,52 +85,66 @@ def ncu_traffic():
 
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clock, power and clock-event reasons through NVML from a background thread
+    (every ~2 ms) while the timed region runs. The device is matched by PCI bus id."""
 
-    def __init__(self, gpu_index: int):
-        self.idx = gpu_index
-        self.proc = None
+    REASONS = (("hw_slowdown", 0x08), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x04), ("hw_power_brake_slowdown", 0x80))
+
+    def __init__(self, device):
+        self.device = device
+        self.rows = []
+        self.err = None
+        self._stop = None
+
+    def _handle(self, nv):
+        p = torch.cuda.get_device_properties(self.device)
+        bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+        return nv.nvmlDeviceGetHandleByPciBusId(bus.encode())
 
     def __enter__(self):
+        import threading
+
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except Exception:
-            self.proc = None
+            import pynvml as nv
+
+            nv.nvmlInit()
+            self.nv = nv
+            self.h = self._handle(nv)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: the line says so
+            self.err = f"nvml unavailable: {e}"
+            return self
+        self._stop = threading.Event()
+
+        def run():
+            nv, h = self.nv, self.h
+            while not self._stop.is_set():
+                try:
+                    self.rows.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                      nv.nvmlDeviceGetCurrentClocksEventReasons(h),
+                                      nv.nvmlDeviceGetPowerUsage(h) / 1000.0))
+                except Exception as e:
+                    self.err = str(e)
+                    return
+                time.sleep(0.002)
+
+        self._t = threading.Thread(target=run, daemon=True)
+        self._t.start()
         return self
 
     def __exit__(self, *a):
-        self.out = ""
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.out, _ = self.proc.communicate(timeout=5)
-            except Exception:
-                self.proc.kill()
+        if self._stop is not None:
+            self._stop.set()
+            self._t.join(timeout=5)
 
     def summary(self):
-        rows = []
-        for line in (self.out or "").splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
-            except ValueError:
-                continue
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        seen = set()
-        for _, _, flags in rows:
-            for n, f in zip(names, flags):
-                if f.lower() == "active":
-                    seen.add(n)
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": sorted(seen), "samples": len(rows)}
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err or "unsampled"]}
+        seen = sorted({n for _, r, _ in self.rows for n, bit in self.REASONS if r & bit})
+        return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": self.max_mhz,
+                "reasons": seen, "samples": len(self.rows), "power_w_max": max(r[2] for r in self.rows),
+                "source": "nvml"}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -198,7 +211,7 @@ def run_ours(args, rank, world, device):
     step_ev, kern = [], []
     barrier()
     torch.cuda.synchronize(device)
-    with ClockSampler(device.index if device.index is not None else 0) as clk:
+    with ClockSampler(device) as clk:
         with torch.cuda.stream(stream):
             for _ in range(args.steps):
                 flush.zero_()
@@ -267,7 +280,7 @@ def run_ours(args, rank, world, device):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     total_ms, q_ms, g_ms, e2e_ms = t.tolist()
     return dict(total_ms=total_ms, q_ms=q_ms, g_ms=g_ms, e2e_ms=e2e_ms, per_proj=per_proj, clocks=clocks,
-                h2d=h2d, d2h=d2h, launches=args.steps * len(PROJ) * 4)
+                h2d=h2d, d2h=d2h, launches=args.steps * len(PROJ) * 2)
 
 
 # ---------------------------------------------------------------------------------------------

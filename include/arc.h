@@ -89,7 +89,8 @@ int64_t arc_kpad(int64_t k_aug);
 size_t arc_nvfp4_codes_bytes(int64_t rows, int64_t k_aug);
 /* Bytes of the swizzled scale bytes: ceil(rows/128) * (K_pad/64) * 512. */
 size_t arc_nvfp4_sf_bytes(int64_t rows, int64_t k_aug);
-/* Workspace of arc_quantize_act_nvfp4 / arc_pack_weight_nvfp4 for `rows` rows and r channels. */
+/* Workspace of arc_quantize_act_nvfp4 / arc_pack_weight_nvfp4 for `rows` rows and r channels:
+ * 8 KiB of per-CTA abs-max partials plus 8 bytes per row (RMSNorm statistics). */
 size_t arc_quantize_workspace_bytes(int64_t rows, int32_t r);
 /* Workspace of arc_calibrate_outliers for K channels. */
 size_t arc_calibrate_workspace_bytes(int64_t K);
@@ -114,7 +115,9 @@ size_t arc_calibrate_workspace_bytes(int64_t K);
  *   d_scale_out     device fp32 scalar receiving the tensor scale used (may equal d_static_scale).
  *   workspace       device scratch of arc_quantize_workspace_bytes(M, r) bytes, 256-byte aligned;
  *                   contents need not be initialised; calls sharing a workspace must be ordered.
- * Requires K % 16 == 0, r % 16 == 0, 0 <= r <= K, ldx >= K, x rows 16-byte aligned.
+ * Requires K % 16 == 0, r % 16 == 0, 0 <= r <= K, ldx >= K, x rows 16-byte aligned. The
+ * residuals are staged in shared memory (about 210 bytes per outlier channel), which accepts
+ * r <= 896 for any K <= 65536; larger requests return ARC_ERR_UNSUPPORTED.
  */
 arc_status arc_quantize_act_nvfp4(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, const int32_t* d_idx,
                                   int32_t r, const void* rms_gain_bf16, float rms_eps, const float* d_static_scale,
@@ -266,8 +269,8 @@ arc_status arc_debug_inject(int32_t kind);
  * `ws_bytes`; the call allocates nothing. Its temporary space is one array of
  * ARC_STATIC_SCRATCH_BYTES bytes of device memory compiled into this library, so every GPU that
  * loads the library holds that array until the process exits.
- *   Limit: arc_quantize_workspace_bytes(M, r) <= ARC_STATIC_SCRATCH_BYTES (for example M = 4096
- *          with r <= 256, or M = 16384 with r <= 64); larger requests return ARC_ERR_WORKSPACE
+ *   Limit: arc_quantize_workspace_bytes(M, r) <= ARC_STATIC_SCRATCH_BYTES, that is 8 KiB plus
+ *          8 bytes per row: up to about 580 000 rows; larger requests return ARC_ERR_WORKSPACE
  *          before any launch.
  *   Set-up: the first call on a device looks up the array's device address on that device (it
  *          must be the current device); make that first call before any stream capture.

@@ -1,5 +1,5 @@
 // arc_device.cuh -- device-side building blocks for sm_100a: status word, bounded waits,
-// mbarriers, TMA and bulk copies, tcgen05 (TMEM allocation, MMA, copies, loads), and the
+// mbarriers, TMA and bulk copies, tcgen05 (TMEM allocation, MMA, loads and stores), and the
 // element codecs of the NVFP4 block format.
 #pragma once
 
@@ -153,21 +153,6 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
   d |= static_cast<uint64_t>(1u) << 46;          // descriptor version for sm_100
   d |= static_cast<uint64_t>(2u) << 61;          // 128-byte swizzle
   return d;
-}
-
-// Descriptor of one 512-byte scale-factor atom as the source of tcgen05.cp 32x128b:
-// 32 rows of 16 bytes, no swizzle, 8-row core matrices 128 bytes apart.
-__device__ __forceinline__ uint64_t desc_sf_atom(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>(128u >> 4) << 32;
-  d |= static_cast<uint64_t>(1u) << 46;
-  return d;
-}
-
-// 32 lanes x 128 bits from shared memory, replicated into all four 32-lane quarters of TMEM.
-__device__ __forceinline__ void tc_cp_sf_atom(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,

@@ -56,10 +56,10 @@ arc_status device_check(int* sms) {
                              arc::gemm_smem_bytes<false>()) != cudaSuccess ||
         cudaFuncSetAttribute(arc::k_gemm<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              arc::gemm_smem_bytes<false>()) != cudaSuccess ||
-        cudaFuncSetAttribute(arc::k_quant_fused<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             arc::kFusedSmem) != cudaSuccess ||
-        cudaFuncSetAttribute(arc::k_quant_fused<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             arc::kFusedSmem) != cudaSuccess)
+        cudaFuncSetAttribute(arc::k_quant_rows<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             arc::kQRowsSmemMax) != cudaSuccess ||
+        cudaFuncSetAttribute(arc::k_quant_rows<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             arc::kQRowsSmemMax) != cudaSuccess)
       return ARC_ERR_CUDA;
     d.attrs_set = true;
   }
@@ -114,36 +114,21 @@ int take_inject() {
 // Quantization driver shared by activations and weights
 // ---------------------------------------------------------------------------------------------
 
-// Quantizer workspace: per-CTA abs-max partials | grid-barrier words (two go words, two arrival
-// words per CTA) | residual stash [r, rows] fp32 | 1/rms per row (double). Nothing in it needs
-// to be initialised.
+// Quantizer workspace: per-CTA abs-max partials | 1/rms per row (double, RMSNorm prologue only).
+// Nothing in it needs to be initialised.
 struct QuantWs {
   uint32_t* partials;
-  unsigned long long* flags;
-  float* stash;
   double* inv_rms;
 };
 
 constexpr int64_t kPartialBytes = arc::kMaxPartials * 4;
-constexpr int64_t kFlagBytes = arc::kMaxPartials * 2 * 8;
 
-QuantWs carve_quant_ws(void* ws, int64_t rows, int32_t r) {
+QuantWs carve_quant_ws(void* ws) {
   uint8_t* b = static_cast<uint8_t*>(ws);
   QuantWs w;
   w.partials = reinterpret_cast<uint32_t*>(b);
-  w.flags = reinterpret_cast<unsigned long long*>(b + kPartialBytes);
-  w.stash = reinterpret_cast<float*>(b + kPartialBytes + kFlagBytes);
-  w.inv_rms =
-      reinterpret_cast<double*>(b + kPartialBytes + kFlagBytes + align256(rows * static_cast<int64_t>(r) * 4));
+  w.inv_rms = reinterpret_cast<double*>(b + kPartialBytes);
   return w;
-}
-
-// Barrier epochs: never reused within a process; the start is taken from the clock so that flags
-// left in recycled device memory by an earlier process do not match.
-unsigned long long next_epoch() {
-  static std::atomic<unsigned long long> counter{
-      (static_cast<unsigned long long>(std::chrono::steady_clock::now().time_since_epoch().count()) << 8) | 1ull};
-  return counter.fetch_add(2);
 }
 
 arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, const int32_t* idx, int32_t r,
@@ -152,7 +137,9 @@ arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, con
   if (!x || !codes || !sf || !scale_out) return ARC_ERR_INVALID_ARG;
   if (M <= 0 || K <= 0 || K % 16 || r < 0 || r % 16 || r > K || ldx < K) return ARC_ERR_INVALID_ARG;
   if (r > 0 && !idx) return ARC_ERR_INVALID_ARG;
-  if (M > (1ll << 30) || K > (1ll << 24)) return ARC_ERR_UNSUPPORTED;
+  if (M > (1ll << 30) || K > (1ll << 20) || r > 32767) return ARC_ERR_UNSUPPORTED;
+  const size_t smem = arc::qrows_smem_bytes(static_cast<int>(K), r);
+  if (smem > static_cast<size_t>(arc::kQRowsSmemMax)) return ARC_ERR_UNSUPPORTED;
   if (!al16(x) || (ldx * 2) % 16 || !al16(codes) || !al16(sf) || (gain && !al16(gain))) return ARC_ERR_ALIGNMENT;
   if (!workspace || ws_bytes < arc_quantize_workspace_bytes(M, r)) return ARC_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ARC_ERR_ALIGNMENT;
@@ -160,18 +147,26 @@ arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, con
   arc_status st = device_check(&sms);
   if (st != ARC_OK) return st;
   cudaStream_t s = S(stream);
-  QuantWs w = carve_quant_ws(workspace, M, r);
-  const double eps_d = static_cast<double>(eps);
+  QuantWs w = carve_quant_ws(workspace);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   const __nv_bfloat16* gb = static_cast<const __nv_bfloat16*>(gain);
   int npartials = 0;
+  bool first = false;
   if (gain) {
     // RMSNorm statistics (and, with a dynamic scale, the abs-max of the normalised rows) first
     npartials = static_cast<int>(std::min<int64_t>((M + 7) / 8, arc::kMaxPartials));
     arc::k_row_stats<<<static_cast<unsigned>(npartials), 256, 0, s>>>(xb, ldx, static_cast<int>(M),
-                                                                     static_cast<int>(K), gb, eps_d, w.inv_rms,
-                                                                     static_scale ? nullptr : w.partials);
+                                                                     static_cast<int>(K), gb, static_cast<double>(eps),
+                                                                     w.inv_rms, static_scale ? nullptr : w.partials);
     if ((st = launch_status()) != ARC_OK) return st;
+    first = true;
+  } else if (!static_scale) {
+    const int64_t items = M * ((K + arc::kAmaxSeg - 1) / arc::kAmaxSeg);
+    npartials = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((items + 7) / 8, arc::kMaxPartials)));
+    arc::k_amax<<<static_cast<unsigned>(npartials), 256, 0, s>>>(xb, ldx, static_cast<int>(M), static_cast<int>(K),
+                                                                w.partials);
+    if ((st = launch_status()) != ARC_OK) return st;
+    first = true;
   }
   QuantArgs a;
   a.x = xb;
@@ -190,38 +185,29 @@ arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, con
   a.scale_out = scale_out;
   a.codes = codes;
   a.sf = sf;
-  a.stash = w.stash;
   a.dup = dup;
-  CUtensorMap tmx;
-  if (!make_map(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
-                static_cast<uint64_t>(ldx * 2), 64, 128))
-    return ARC_ERR_CUDA;
-  const int tiles_k = static_cast<int>((K + 127) / 128);
-  const int ntiles = static_cast<int>((M + 127) / 128) * tiles_k;
-  // one resident CTA per SM: the launch is cooperative, so every CTA runs at once and the grid
-  // barriers inside the kernel are safe
+  const int mpad = static_cast<int>((M + 127) / 128 * 128);
+  const void* kern = gain ? reinterpret_cast<const void*>(arc::k_quant_rows<true>)
+                          : reinterpret_cast<const void*>(arc::k_quant_rows<false>);
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gain ? arc::k_quant_fused<true> : arc::k_quant_fused<false>,
-                                                    arc::kFusedThreads, arc::kFusedSmem) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, arc::kQRowThreads, smem) != cudaSuccess ||
       per_sm < 1)
     return ARC_ERR_CUDA;
-  // the barrier words hold two go words (256 bytes) and two arrival words per CTA
-  const int grid = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(ntiles), static_cast<int64_t>(sms) * per_sm,
-                                                        static_cast<int64_t>(arc::kMaxPartials - 16)}));
-  arc::FusedArgs f;
-  f.tiles_k = tiles_k;
-  f.ntiles = ntiles;
-  f.do_amax = (!gain && !static_scale) ? 1 : 0;
-  f.partials = w.partials;
-  f.flags = w.flags;
-  f.epoch = next_epoch();
-  f.wait_ns = g_wait_ns;
-  f.mpad = static_cast<int>((M + 127) / 128 * 128);
-  void* args[] = {&tmx, &a, &f};
-  const cudaError_t e =
-      cudaLaunchCooperativeKernel(gain ? reinterpret_cast<const void*>(arc::k_quant_fused<true>)
-                                       : reinterpret_cast<const void*>(arc::k_quant_fused<false>),
-                                  dim3(grid), dim3(arc::kFusedThreads), args, arc::kFusedSmem, s);
+  const int64_t want = mpad;  // one row per CTA at a time
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(want, static_cast<int64_t>(sms) * per_sm));
+  // the second launch may begin while the first one runs; it waits for the first one's results
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(arc::kQRowThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = first ? 1 : 0;
+  const cudaError_t e = gain ? cudaLaunchKernelEx(&cfg, arc::k_quant_rows<true>, a, mpad)
+                             : cudaLaunchKernelEx(&cfg, arc::k_quant_rows<false>, a, mpad);
   return e == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
 }
 
@@ -277,8 +263,7 @@ size_t arc_nvfp4_sf_bytes(int64_t rows, int64_t k_aug) {
 
 size_t arc_quantize_workspace_bytes(int64_t rows, int32_t r) {
   if (rows < 0 || r < 0) return 0;
-  return static_cast<size_t>(kPartialBytes + kFlagBytes + align256(rows * static_cast<int64_t>(r) * 4) +
-                             align256(rows * 8));
+  return static_cast<size_t>(kPartialBytes + align256(rows * 8));
 }
 
 size_t arc_calibrate_workspace_bytes(int64_t K) {

@@ -8,24 +8,19 @@
 // each outlier channel, x - E2M1(code)*d, is quantized again with the same tensor scale and
 // appended after the K primary channels (weights append the channel itself).
 //
-// Work split:
-//   k_row_stats    one warp per row: exact sum of squares -> 1/rms (double); with a dynamic
-//                  scale also max |RMSNorm(x)|, one partial per CTA
-//   k_quant_fused  one cooperative launch, one CTA per SM, tiles of 128 rows x 128 channels
-//                  TMA-loaded into a ring of shared-memory buffers by a producer warp, which
-//                  also lists each tile's outlier channels; sixteen coding warps take the tiles
-//                  (full/empty mbarriers between the two roles):
-//     phase 1  (dynamic scale without RMSNorm) max |x| over the CTA's tiles, the last ones
-//              staying resident in the ring; grid barrier; every CTA reduces the partials
-//     phase 2  code the tiles (resident ones first): each coding warp takes eight rows of a
-//              tile, one lane per 16-element block; codes and scale bytes go straight to
-//              global memory; then the warp stashes the residuals of the outlier channels
-//              of its rows in the column-major stash [r, M] (one (row, outlier) pair per
-//              lane, operands fetched by warp shuffles); the warps never wait for one
-//              another, only for tiles
-//     phase 3  after a second grid barrier: the appended residual blocks and the zero
-//              padding up to K_pad, one lane per (row, block) with rows fastest, so the
-//              stash reads are coalesced
+// Work split (two launches, the second started early through programmatic dependent launch so
+// that its set-up overlaps the first):
+//   k_amax        (dynamic scale, no RMSNorm) streams X once: max |x|, one partial per CTA
+//   k_row_stats   (RMSNorm prologue) one warp per row: exact sum of squares -> 1/rms (double);
+//                 with a dynamic scale also max |RMSNorm(x)|, one partial per CTA
+//   k_quant_rows  one CTA per row at a time, every thread four 16-element blocks in flight: block scale,
+//                 E2M1 codes, scale byte (four neighbouring lanes' bytes gathered into one
+//                 32-bit store in the swizzled layout); once the row's K channels are done, the
+//                 CTA forms the residual (activations) or value (weights) of each outlier
+//                 channel from the blocks holding outliers, which the coding threads kept in
+//                 shared memory (values, codes, d), stages them in its stash, codes the r/16
+//                 appended blocks and zero-fills the padding up to K_pad. A row never leaves its warp, so no grid-wide
+//                 synchronisation is needed.
 // Divisions are correctly rounded: x/d is formed as the negated quotient from -RN(1/d) with one
 // exact-remainder correction (Markstein), which keeps the sign of zero quotients, and the codes
 // of the negated quotients have their sign bits flipped back; a plain IEEE divide is used when
@@ -51,7 +46,6 @@ struct QuantArgs {
   float* scale_out;
   uint8_t* codes;
   uint8_t* sf;
-  float* stash;  // [r, M]: column j holds channel idx[j] of every row
   int dup;       // 1: weights (stash the value itself), 0: activations (stash the residual)
 };
 
@@ -94,6 +88,19 @@ __device__ __forceinline__ int64_t sf_offset(int64_t m, int64_t kb, int katoms) 
   return ((m >> 7) * katoms + (kb >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (kb & 3);
 }
 
+// Rare paths kept out of line so the hot loops stay small: plain IEEE divides for operands
+// outside [2^-90, 2^90], where the reciprocal-based forms could under- or overflow.
+__device__ __noinline__ float block_t_slow(float amax, float s) { return __fdiv_rn(__fdiv_rn(amax, 6.0f), s); }
+__device__ __noinline__ uint2 encode16_slow(float d, float x0, float x1, float x2, float x3, float x4, float x5,
+                                            float x6, float x7, float x8, float x9, float x10, float x11, float x12,
+                                            float x13, float x14, float x15) {
+  const float lo[8] = {__fdiv_rn(x0, d), __fdiv_rn(x1, d), __fdiv_rn(x2, d), __fdiv_rn(x3, d),
+                       __fdiv_rn(x4, d), __fdiv_rn(x5, d), __fdiv_rn(x6, d), __fdiv_rn(x7, d)};
+  const float hi[8] = {__fdiv_rn(x8, d),  __fdiv_rn(x9, d),  __fdiv_rn(x10, d), __fdiv_rn(x11, d),
+                       __fdiv_rn(x12, d), __fdiv_rn(x13, d), __fdiv_rn(x14, d), __fdiv_rn(x15, d)};
+  return make_uint2(e2m1x8_rn_sat(lo), e2m1x8_rn_sat(hi));
+}
+
 // Scale byte and decode scale d of a block with abs-max `amax` under tensor scale s:
 // t = (amax / 6) / s (two correctly rounded divides), sf = E4M3(t), d = E4M3value(sf) * s.
 __device__ __forceinline__ uint32_t block_scale(float amax, float s, float rcp_s, float rcp6, float* d) {
@@ -104,11 +111,45 @@ __device__ __forceinline__ uint32_t block_scale(float amax, float s, float rcp_s
     // outside [2^-20, 2^20] the E4M3 result is 0 or 448 whatever the last bit of t
     t = (q0 >= 9.5367431640625e-07f && q0 <= 1048576.0f) ? div_rn_from_rcp(t1, s, rcp_s) : q0;
   } else {
-    t = __fdiv_rn(__fdiv_rn(amax, 6.0f), s);
+    t = block_t_slow(amax, s);
   }
   const uint32_t sfb = e4m3_rn_sat(t);
   *d = __fmul_rn(e4m3_value(sfb), s);
   return sfb;
+}
+
+// Scale byte of a block with abs-max `amax` under tensor scale s: E4M3((amax / 6) / s), two
+// correctly rounded divides (the decode scale is then E4M3value(byte) * s).
+__device__ __forceinline__ uint32_t block_sf(float amax, float s, float rcp_s, float rcp6) {
+  float t;
+  if (in_safe_range(amax) && in_safe_range(s)) {
+    const float t1 = div_rn_from_rcp(amax, 6.0f, rcp6);
+    const float q0 = __fmul_rn(t1, rcp_s);
+    t = (q0 >= 9.5367431640625e-07f && q0 <= 1048576.0f) ? div_rn_from_rcp(t1, s, rcp_s) : q0;
+  } else {
+    t = block_t_slow(amax, s);
+  }
+  return e4m3_rn_sat(t);
+}
+
+// Codes of 16 values against decode scale d > 0 with nrcp = -RN(1/d) taken from a table (0 when
+// d is outside the range where the reciprocal form is exact): same result as encode16.
+__device__ __forceinline__ uint2 encode16_nr(const uint64_t (&p)[8], float d, float nrcp) {
+  if (nrcp == 0.0f) {
+    float x[16];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f2_unpack(p[j], x[2 * j], x[2 * j + 1]);
+    return encode16_slow(d, x[0], x[1], x[2], x[3], x[4], x[5], x[6], x[7], x[8], x[9], x[10], x[11], x[12],
+                         x[13], x[14], x[15]);
+  }
+  float lo[8], hi[8];
+  const uint64_t nrcp2 = f2_pack(nrcp, nrcp), d2 = f2_pack(d, d);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    f2_unpack(neg_div2_rn(p[j], d2, nrcp2), lo[2 * j], lo[2 * j + 1]);
+    f2_unpack(neg_div2_rn(p[4 + j], d2, nrcp2), hi[2 * j], hi[2 * j + 1]);
+  }
+  return make_uint2(e2m1x8_rn_sat(lo) ^ 0x88888888u, e2m1x8_rn_sat(hi) ^ 0x88888888u);
 }
 
 // Codes of 16 values (8 packed pairs) against decode scale d > 0: E2M1 of the correctly rounded
@@ -117,21 +158,19 @@ __device__ __forceinline__ uint32_t block_scale(float amax, float s, float rcp_s
 // with symmetric rounding and saturation, code(q) = code(-q) ^ 8 nibble by nibble. Element i of
 // pair j in bits 8j + 4i.
 __device__ __forceinline__ uint2 encode16(const uint64_t (&p)[8], float d) {
-  float nq[16];
-  if (in_safe_range(d)) {
-    const float nrcp = -__frcp_rn(d);
-    const uint64_t nrcp2 = f2_pack(nrcp, nrcp), d2 = f2_pack(d, d);
+  if (!in_safe_range(d)) {
+    float x[16];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) f2_unpack(neg_div2_rn(p[j], d2, nrcp2), nq[2 * j], nq[2 * j + 1]);
-  } else {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      float x0, x1;
-      f2_unpack(p[j], x0, x1);
-      nq[2 * j] = -__fdiv_rn(x0, d);
-      nq[2 * j + 1] = -__fdiv_rn(x1, d);
-    }
+    for (int j = 0; j < 8; ++j) f2_unpack(p[j], x[2 * j], x[2 * j + 1]);
+    // the hardware conversion keeps the sign of a zero quotient, like the negated fast path
+    return encode16_slow(d, x[0], x[1], x[2], x[3], x[4], x[5], x[6], x[7], x[8], x[9], x[10], x[11], x[12],
+                         x[13], x[14], x[15]);
   }
+  float nq[16];
+  const float nrcp = -__frcp_rn(d);
+  const uint64_t nrcp2 = f2_pack(nrcp, nrcp), d2 = f2_pack(d, d);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) f2_unpack(neg_div2_rn(p[j], d2, nrcp2), nq[2 * j], nq[2 * j + 1]);
   float lo[8], hi[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -236,6 +275,7 @@ __device__ double warp_row_inv_rms(const __nv_bfloat16* __restrict__ h, int K, d
 __global__ void __launch_bounds__(256) k_row_stats(const __nv_bfloat16* __restrict__ h, int64_t ldh, int M, int K,
                                                    const __nv_bfloat16* __restrict__ gain, double eps,
                                                    double* inv_rms, uint32_t* partials) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the quantizer may start early
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint32_t mx = 0;
   for (int m = blockIdx.x * 8 + warp; m < M; m += gridDim.x * 8) {
@@ -260,402 +300,260 @@ __global__ void __launch_bounds__(256) k_row_stats(const __nv_bfloat16* __restri
 }
 
 // ---------------------------------------------------------------------------------------------
-// Single-launch quantizer (cooperative launch, one CTA per SM, all CTAs resident).
-// The grid barriers need no initialised memory: each CTA stores the call's epoch (a number the
-// host never reuses) in its own flag and waits until every flag shows it, with the usual time
-// limit; a wait that runs out sets the status word and stops the CTA.
-// ---------------------------------------------------------------------------------------------
-constexpr int kQTileBytes = 128 * 128 * 2;  // one X tile: two TMA boxes of 128 rows x 64 channels
-constexpr int kCodeWarps = 16;                      // warps that code tiles
-constexpr int kFusedThreads = (kCodeWarps + 1) * 32;  // plus one producer warp (loads, outlier lists)
-constexpr int kFusedBufs = 6;
-constexpr int kIdxSmem = 1024;  // outlier indices kept in shared memory (the rest read from L2)
-// dynamic shared memory: the ring of X tiles, 1024-aligned for the 128-byte swizzle
-constexpr int kFusedSmem = 1024 + kFusedBufs * kQTileBytes;
+// Programmatic dependent launch: the quantizer's second kernel may start while the first one
+// runs; it waits here before it reads the first one's results.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// Grid barrier over co-resident CTAs: each CTA publishes the call's epoch in its own arrival
-// word; CTA 0 gathers them (one polling thread per word) and then publishes the epoch in the
-// go word, which one thread of every CTA polls. Polling from every CTA on every arrival word
-// crowds a few L2 lines with requests and costs about twice as much. Release stores and acquire
-// loads at GPU scope carry each CTA's earlier writes (made visible to thread 0 by the CTA
-// barrier) to every CTA after the barrier. Every wait is bounded; one that runs out sets the
-// status word and makes the barrier return false in every CTA that sees it.
-__device__ __forceinline__ bool grid_barrier(unsigned long long* arrive, unsigned long long* go, int G,
-                                             unsigned long long epoch, uint64_t wait_ns, int* abort_sh) {
-  __syncthreads();
-  if (threadIdx.x == 0) st_release_gpu(&arrive[blockIdx.x], epoch);
-  const uint64_t t0 = globaltimer_ns();
-  bool ok = true;
-  if (blockIdx.x == 0) {
-    for (int i = threadIdx.x; i < G && ok; i += blockDim.x)
-      while (ld_acquire_gpu(&arrive[i]) != epoch) {
-        if (globaltimer_ns() - t0 > wait_ns) {
-          ok = false;
-          break;
-        }
-      }
-    ok = __syncthreads_and(ok);
-    if (threadIdx.x == 0 && ok) st_release_gpu(go, epoch);
-  }
-  if (threadIdx.x == 0 && ok) {
-    while (ld_acquire_gpu(go) != epoch) {
-      if (globaltimer_ns() - t0 > wait_ns) {
-        ok = false;
-        break;
-      }
-    }
-  }
-  if (!ok) {
-    set_status(kStatusTimeout);
-    *reinterpret_cast<volatile int*>(abort_sh) = 1;
-  }
-  __syncthreads();
-  return *reinterpret_cast<volatile int*>(abort_sh) == 0;
-}
+constexpr int kAmaxSeg = 2048;  // elements of a row per warp work item
 
-struct FusedArgs {
-  int tiles_k, ntiles;
-  int do_amax;                  // phase 1 runs (dynamic scale without RMSNorm)
-  uint32_t* partials;           // [gridDim.x] written by phase 1
-  unsigned long long* flags;    // barrier words: go words at [0] and [16], arrivals at [32 ..)
-  unsigned long long epoch;     // this call's barrier epochs: epoch and epoch + 1
-  uint64_t wait_ns;
-  int mpad;                     // rows rounded up to 128 (scale padding rows)
-};
-
-// Shared-memory address of 16-byte chunk j (0..7) of tile row `row` in half h (channels
-// 64h .. 64h+63): each half is 128 rows x 128 bytes with the 128-byte swizzle.
-__device__ __forceinline__ uint32_t qtile_chunk(uint32_t base, int h, int row, int j) {
-  return base + h * (128 * 128) + row * 128 + ((j ^ (row & 7)) << 4);
-}
-
-// Outlier list of one column tile: entries (j << 7) | (channel - k0) for the index-list
-// positions j whose channel falls in the tile, in increasing j.
-constexpr int kOCap = 256;  // entries per tile (128 distinct channels at most)
-struct OutlierList {
-  int n;
-  uint32_t e[kOCap];
-};
-
-// Codes of one resident tile, by one coding warp: lane l takes row 8w + l%8 and blocks l/8 and
-// 4 + l/8 of it (eight rows per 16-byte read hit eight distinct swizzled bank groups, and each
-// code store is 32 contiguous bytes in each of eight rows). Both blocks are loaded first and
-// coded side by side, and the lane writes its codes and scale bytes. Then the warp stashes the
-// outlier channels of its eight rows: lane l takes row l%8 and outlier entry l/8 (four entries
-// per pass), fetching the decode scale and code word of that element from the lane that coded
-// it by warp shuffles, and writes x (weights) or x minus its dequantized value (activations) to
-// column j of the stash. Nothing here waits for another warp.
-//   sf_lane: this lane's constant part of the scale offset, (mm%32)*16 + (mm/32)*4 + l/8
-template <bool RMS>
-__device__ __forceinline__ void code_rows(const QuantArgs& a, uint32_t tbase, int tm, int tk, float s, float rcp_s,
-                                          float rcp6, const OutlierList& ol, int sf_lane) {
+// max |x| over X [M, K]: warps over (row, 2048-element segment) items, eight 16-byte loads in
+// flight per lane; one partial per CTA (fp32 bits of the magnitude).
+__global__ void __launch_bounds__(256) k_amax(const __nv_bfloat16* __restrict__ x, int64_t ldx, int M, int K,
+                                              uint32_t* partials) {
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mm = warp * 8 + (lane & 7), bq = lane >> 3;
-  const int m0 = tm * 128, k0 = tk * 128;
-  const int m = m0 + mm;
-  const bool rowok = m < a.M;
-  double inv = 0.0;
-  if (RMS) inv = rowok ? a.inv_rms[m] : 0.0;
-  uint32_t ws[2][8];
+  const int nseg = (K + kAmaxSeg - 1) / kAmaxSeg;
+  const int64_t items = static_cast<int64_t>(M) * nseg;
+  uint32_t mx = 0;
+  for (int64_t it = static_cast<int64_t>(blockIdx.x) * 8 + warp; it < items; it += static_cast<int64_t>(gridDim.x) * 8) {
+    const int m = static_cast<int>(it / nseg), seg = static_cast<int>(it - static_cast<int64_t>(m) * nseg);
+    const __nv_bfloat16* row = x + static_cast<int64_t>(m) * ldx;
+    const int k0 = seg * kAmaxSeg + 8 * lane;
+    const int k1 = min(K, (seg + 1) * kAmaxSeg);
+    uint4 w[8];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const uint4 w0 = lds_v4(qtile_chunk(tbase, h, mm, 2 * bq));
-    const uint4 w1 = lds_v4(qtile_chunk(tbase, h, mm, 2 * bq + 1));
-    ws[h][0] = w0.x, ws[h][1] = w0.y, ws[h][2] = w0.z, ws[h][3] = w0.w;
-    ws[h][4] = w1.x, ws[h][5] = w1.y, ws[h][6] = w1.z, ws[h][7] = w1.w;
+    for (int i = 0; i < 8; ++i) w[i] = (k0 + 256 * i < k1) ? ld_nc_v4(row + k0 + 256 * i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx = absmax_bf16x2(mx, w[i]);
   }
-  float v[2][16];
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int kcol = k0 + 16 * (4 * h + bq);
-    if (RMS) {
-      uint4 g0 = make_uint4(0, 0, 0, 0), g1 = g0;
-      if (kcol < a.K) {
-        g0 = ld_nc_v4(a.gain + kcol);
-        g1 = ld_nc_v4(a.gain + kcol + 8);
-      }
-      const uint32_t gs[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        v[h][2 * j] = rms_apply(bf16_lo(ws[h][j]), inv, bf16_lo(gs[j]));
-        v[h][2 * j + 1] = rms_apply(bf16_hi(ws[h][j]), inv, bf16_hi(gs[j]));
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        v[h][2 * j] = bf16_lo(ws[h][j]);
-        v[h][2 * j + 1] = bf16_hi(ws[h][j]);
-      }
-    }
-  }
-  float d[2];
-  uint32_t sfv[2];
-  uint2 codes[2];
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const float a0 = fmax3_abs(v[h][0], v[h][1], v[h][2]), a1 = fmax3_abs(v[h][3], v[h][4], v[h][5]),
-                a2 = fmax3_abs(v[h][6], v[h][7], v[h][8]), a3 = fmax3_abs(v[h][9], v[h][10], v[h][11]),
-                a4 = fmax3_abs(v[h][12], v[h][13], v[h][14]);
-    sfv[h] = block_scale(fmaxf(fmax3(a0, a1, a2), fmax3(a3, a4, fabsf(v[h][15]))), s, rcp_s, rcp6, &d[h]);
-  }
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    uint64_t p[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) p[j] = f2_pack(v[h][2 * j], v[h][2 * j + 1]);
-    codes[h] = (d[h] == 0.0f) ? make_uint2(0u, 0u) : encode16(p, d[h]);
-  }
-  uint8_t* crow = a.codes + static_cast<int64_t>(rowok ? m : 0) * (a.kpad >> 1) + (k0 >> 1);
-  uint8_t* sft = a.sf + (static_cast<int64_t>(tm) * a.katoms + (k0 >> 6)) * 512 + sf_lane;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    if (k0 + 16 * (4 * h + bq) >= a.K) continue;
-    if (rowok) *reinterpret_cast<uint2*>(crow + 8 * (4 * h + bq)) = codes[h];
-    // padding rows (up to the next multiple of 128) carry zero scales
-    sft[h * 512] = rowok ? static_cast<uint8_t>(sfv[h]) : 0;
-  }
-  // outlier channels of the warp's eight rows, four entries per pass (the lane keeps its row)
-  for (int base = 0; base < ol.n; base += 4) {
-    const int o = base + (lane >> 3);
-    const bool act = o < ol.n && rowok;
-    const uint32_t ent = (o < ol.n) ? ol.e[o] : 0u;
-    const int col = static_cast<int>(ent & 127u), j = static_cast<int>(ent >> 7);
-    const int blk = col >> 4, e = col & 15;
-    const int src = (lane & 7) + 8 * (blk & 3);  // the lane that coded (this row, block blk)
-    const float dd0 = __shfl_sync(0xFFFFFFFFu, d[0], src), dd1 = __shfl_sync(0xFFFFFFFFu, d[1], src);
-    const uint32_t c0x = __shfl_sync(0xFFFFFFFFu, codes[0].x, src), c0y = __shfl_sync(0xFFFFFFFFu, codes[0].y, src);
-    const uint32_t c1x = __shfl_sync(0xFFFFFFFFu, codes[1].x, src), c1y = __shfl_sync(0xFFFFFFFFu, codes[1].y, src);
-    if (!act) continue;
-    uint16_t hv;
-    asm volatile("ld.shared.u16 %0, [%1];"
-                 : "=h"(hv)
-                 : "r"(qtile_chunk(tbase, blk >> 2, mm, (col & 63) >> 3) + 2 * (col & 7)));
-    float x = __uint_as_float(static_cast<uint32_t>(hv) << 16);
-    if (RMS) x = rms_apply(x, inv, __bfloat162float(a.gain[k0 + col]));
-    float res = x;
-    if (!a.dup) {
-      const uint32_t cw = (blk >> 2) ? ((e < 8) ? c1x : c1y) : ((e < 8) ? c0x : c0y);
-      const uint32_t c = (cw >> (4 * (e & 7))) & 15u;
-      res = __fsub_rn(x, __fmul_rn(e2m1_value(c), (blk >> 2) ? dd1 : dd0));
-    }
-    a.stash[static_cast<int64_t>(j) * a.M + m] = res;
-  }
+  cta_max_to(max(mx & 0xFFFFu, mx >> 16) << 16, &partials[blockIdx.x]);
 }
 
-// The outlier list of column tile k0 .. k0+127, by one warp (ballot compaction).
-__device__ __forceinline__ void build_olist(const QuantArgs& a, const int32_t* idx_sh, int k0, OutlierList& ol,
-                                            int lane) {
-  int n = 0;
-  for (int base = 0; base < a.r; base += 32) {
-    const int j = base + lane;
-    const int c = (j < a.r) ? (j < kIdxSmem ? idx_sh[j] : __ldg(a.idx + j)) : -1;
-    const bool hit = j < a.r && c < a.K && static_cast<unsigned>(c - k0) < 128u;
-    const uint32_t mask = __ballot_sync(0xFFFFFFFFu, hit);
-    const int pos = n + __popc(mask & ((1u << lane) - 1u));
-    if (hit && pos < kOCap) ol.e[pos] = (static_cast<uint32_t>(j) << 7) | static_cast<uint32_t>(c - k0);
-    n += __popc(mask);
-  }
-  if (n > kOCap) {
-    if (lane == 0) set_status(kStatusInvalidArg);  // more entries than distinct channels
-    n = kOCap;
-  }
-  if (lane == 0) ol.n = n;
-  __syncwarp();
-}
+constexpr int kQRowThreads = 128;  // one CTA codes one row at a time
+constexpr int kQRowDepth = 4;      // 16-element blocks in flight per thread
+constexpr int kQRowsSmemMax = 200 * 1024;  // largest dynamic shared memory the call accepts
 
-// The appended residual blocks (from the stash) and zero padding up to K_pad: one (row, block)
-// per thread, rows fastest.
-__device__ __forceinline__ void tail_items(const QuantArgs& a, int mpad, float s, float rcp_s, float rcp6) {
-  const int nres = a.r >> 4;
-  const int ntail = (a.kpad - a.K) >> 4;
-  const int64_t cpitch = a.kpad >> 1;
-  const int64_t items = static_cast<int64_t>(mpad) * ntail;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t it = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it < items; it += stride) {
-    const int b = static_cast<int>(it / mpad), m = static_cast<int>(it - static_cast<int64_t>(b) * mpad);
-    uint32_t sfv = 0;
-    uint2 codes = make_uint2(0u, 0u);
-    if (m < a.M && b < nres) {
-      const float* src = a.stash + static_cast<int64_t>(16 * b) * a.M + m;
-      float v[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = __ldcg(src + static_cast<int64_t>(i) * a.M);
-      uint64_t p[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) p[j] = f2_pack(v[2 * j], v[2 * j + 1]);
-      const float a0 = fmax3_abs(v[0], v[1], v[2]), a1 = fmax3_abs(v[3], v[4], v[5]),
-                  a2 = fmax3_abs(v[6], v[7], v[8]), a3 = fmax3_abs(v[9], v[10], v[11]),
-                  a4 = fmax3_abs(v[12], v[13], v[14]);
-      const float am = fmaxf(fmax3(a0, a1, a2), fmax3(a3, a4, fabsf(v[15])));
-      float d;
-      sfv = block_scale(am, s, rcp_s, rcp6, &d);
-      if (d != 0.0f) codes = encode16(p, d);
-    }
-    if (m < a.M) *reinterpret_cast<uint2*>(a.codes + static_cast<int64_t>(m) * cpitch + ((a.K + 16 * b) >> 1)) = codes;
-    a.sf[sf_offset(m, (a.K >> 4) + b, a.katoms)] = static_cast<uint8_t>(sfv);
-  }
+// Dynamic shared memory of k_quant_rows:
+//   idx_s     int32 [r]        the outlier channels (-1 for an out-of-range entry)
+//   blk_slot  int16 [K/16]     slot of each 16-channel block holding an outlier, else -1
+//   slots     [nslot]          48 bytes per outlier block of the current row: values, codes, d
+//   stash     float [r]        the row's residuals (values for weights) in idx order
+__host__ __device__ constexpr int qrows_nslot(int K, int r) { return r < K / 16 ? r : K / 16; }
+__host__ __device__ constexpr size_t qrows_smem_bytes(int K, int r) {
+  return (static_cast<size_t>(r) * 4 + 15) / 16 * 16 + (static_cast<size_t>(K / 16) * 2 + 15) / 16 * 16 +
+         static_cast<size_t>(qrows_nslot(K, r)) * 48 + (static_cast<size_t>(r) * 4 + 15) / 16 * 16 + 16;
 }
 
 template <bool RMS>
-__global__ void __launch_bounds__(kFusedThreads, 1) k_quant_fused(const __grid_constant__ CUtensorMap tmX,
-                                                                  QuantArgs a, FusedArgs f) {
-  extern __shared__ uint8_t fsmem_raw[];
-  uint8_t* qs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fsmem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t full[kFusedBufs], empty[kFusedBufs];
-  __shared__ int32_t idx_sh[kIdxSmem];
-  __shared__ OutlierList olist[kFusedBufs];  // outlier list of the tile in each ring buffer
-  __shared__ int abort_sh;
-  __shared__ float s_sh;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool producer = warp == kCodeWarps;
-  const int G = gridDim.x;
-  const int n_c = (f.ntiles > static_cast<int>(blockIdx.x)) ? (f.ntiles - blockIdx.x + G - 1) / G : 0;
-  const uint32_t xbase = smem_u32(qs);
-  // CTA-local tile i is tile blockIdx.x + i * G. Phase 1 streams i = 0 .. n_c-1 through slots
-  // 0 .. n_c-1 and leaves the last `resident` of them in the ring; phase 2 codes those first,
-  // then the others, which come through the ring again. Slot sl uses buffer sl % kFusedBufs.
-  const int resident = f.do_amax ? min(n_c, kFusedBufs) : 0;
-  const int first_slot = f.do_amax ? n_c - resident : 0;  // slot of processing position q = 0
-  auto tile_at = [&](int q) {
-    const int i = f.do_amax ? (q < resident ? n_c - resident + q : q - resident) : q;
-    return static_cast<int>(blockIdx.x) + i * G;
-  };
-  int issued = 0;  // producer lane 0: slots issued so far
-  auto issue = [&](int slot, int t) {
-    const int tm = t / f.tiles_k, tk = t - tm * f.tiles_k;
-    const int buf = slot % kFusedBufs;
-    mbar_arrive_expect_tx(&full[buf], kQTileBytes);
-    uint8_t* dst = qs + buf * kQTileBytes;
-    tma_load_2d(dst, &tmX, &full[buf], tk * 128, tm * 128);
-    tma_load_2d(dst + 128 * 128, &tmX, &full[buf], tk * 128 + 64, tm * 128);
-    issued = slot + 1;
-  };
-  // producer: before reusing a buffer, wait until the coding warps released its previous slot
-  // (sleeping between polls, so the wait leaves the issue slots to the coding warps)
-  auto wait_free = [&](int slot) -> bool {
-    if (slot < kFusedBufs) return true;
-    return mbar_wait(&empty[slot % kFusedBufs], static_cast<uint32_t>((slot / kFusedBufs - 1) & 1), f.wait_ns,
-                     &abort_sh, 128);
-  };
-  // producer lane 0 after an abort: the last load issued into each buffer lands (bounded)
-  auto drain = [&]() {
-    const uint64_t t0 = globaltimer_ns();
-    for (int b = 0; b < kFusedBufs; ++b) {
-      int sl = issued - 1 - ((issued - 1 - b) % kFusedBufs + kFusedBufs) % kFusedBufs;
-      if (sl < 0) continue;
-      while (!mbar_test(&full[b], static_cast<uint32_t>((sl / kFusedBufs) & 1)) && globaltimer_ns() - t0 < f.wait_ns) {
-      }
-    }
-  };
-  auto release = [&](int slot) {  // coding warp done with the slot's buffer and outlier list
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[slot % kFusedBufs]);
-  };
-  // A full barrier completes on the tile's bytes plus two producer arrivals: one with the
-  // byte count when the loads are issued, one when the tile's outlier list is written.
-  if (producer && lane == 0) {
-    for (int i = 0; i < kFusedBufs; ++i) {
-      mbar_init(&full[i], 2);
-      mbar_init(&empty[i], kCodeWarps);
-    }
-    abort_sh = 0;
-    fence_mbar_init();
-    tma_prefetch_desc(&tmX);
-    // the first kFusedBufs slots hold tiles 0 .. kFusedBufs-1 in either phase order
-    for (int sl = 0; sl < min(n_c, kFusedBufs); ++sl) issue(sl, static_cast<int>(blockIdx.x) + sl * G);
-  }
-  for (int j = tid; j < min(a.r, kIdxSmem); j += kFusedThreads) idx_sh[j] = a.idx[j];
-  if (blockIdx.x == 0)
-    for (int j = tid; j < a.r; j += kFusedThreads)
-      if (static_cast<unsigned>(a.idx[j]) >= static_cast<unsigned>(a.K)) set_status(kStatusInvalidArg);
+__global__ void __launch_bounds__(kQRowThreads, 6) k_quant_rows(QuantArgs a, int mpad) {
+  extern __shared__ __align__(16) uint8_t qsm[];
+  const int nblk = a.K >> 4;
+  const int tid = threadIdx.x, lane = tid & 31;
+  constexpr int NT = kQRowThreads;
+  int32_t* idx_s = reinterpret_cast<int32_t*>(qsm);
+  int16_t* blk_slot = reinterpret_cast<int16_t*>(qsm + (static_cast<size_t>(a.r) * 4 + 15) / 16 * 16);
+  uint4* slots = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(blk_slot) +
+                                          (static_cast<size_t>(nblk) * 2 + 15) / 16 * 16);  // 3 x 16 B each
+  float* stash = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(slots) +
+                                          static_cast<size_t>(qrows_nslot(a.K, a.r)) * 48);
+  __shared__ int nslot_sh;
+
+  // outlier tables (before the wait: they overlap the first kernel); out-of-range entries are
+  // reported and left out
+  for (int b = tid; b < nblk; b += NT) blk_slot[b] = -1;
+  if (tid == 0) nslot_sh = 0;
   __syncthreads();
-  if (f.do_amax) {
-    // ------------------------------------------------------------------ phase 1: max |x|
-    uint32_t mx = 0;
-    if (producer) {
-      if (lane == 0) {
-        for (int sl = 0; sl < n_c; ++sl) {
-          if (sl >= kFusedBufs) {
-            if (!wait_free(sl)) break;
-            issue(sl, static_cast<int>(blockIdx.x) + sl * G);
-          }
-          mbar_arrive(&full[sl % kFusedBufs]);  // phase 1 reads no outlier list
-        }
-      }
-      __syncwarp();
-      // outlier lists of the tiles that stay resident (their buffers hold no list in phase 1;
-      // the grid barrier below publishes them)
-      for (int sl = first_slot; sl < n_c; ++sl)
-        build_olist(a, idx_sh, (tile_at(sl - first_slot) % f.tiles_k) * 128, olist[sl % kFusedBufs], lane);
-    } else {
-      for (int sl = 0; sl < n_c; ++sl) {
-        const int buf = sl % kFusedBufs;
-        if (!mbar_wait(&full[buf], static_cast<uint32_t>((sl / kFusedBufs) & 1), f.wait_ns, &abort_sh)) break;
-        const uint32_t tb = xbase + buf * kQTileBytes;
-        // 512 threads x 4 chunks of 16 bytes = the 32 KB tile
-#pragma unroll
-        for (int j = 0; j < 4; ++j) mx = absmax_bf16x2(mx, lds_v4(tb + (tid + j * kCodeWarps * 32) * 16));
-        if (sl < first_slot) release(sl);
-      }
-    }
-    cta_max_to(max(mx & 0xFFFFu, mx >> 16) << 16, &f.partials[blockIdx.x]);
-    if (!grid_barrier(f.flags + 32, f.flags, G, f.epoch, f.wait_ns, &abort_sh)) {
-      if (producer && lane == 0) drain();
-      return;
-    }
+  for (int j = tid; j < a.r; j += NT) {
+    const int c = a.idx[j];
+    const bool ok = static_cast<unsigned>(c) < static_cast<unsigned>(a.K);
+    if (!ok && blockIdx.x == 0) set_status(kStatusInvalidArg);
+    idx_s[j] = ok ? c : -1;
+    if (ok) blk_slot[c >> 4] = -2;
   }
-  // ---------------------------------------------------------------------- phase 2: code tiles
+  __syncthreads();
+  for (int b = tid; b < nblk; b += NT)
+    if (blk_slot[b] == -2) blk_slot[b] = static_cast<int16_t>(atomicAdd(&nslot_sh, 1));
+
+  // ---- tensor scale
+  pdl_wait();
+  float s;
   {
-    QuantArgs aa = a;
-    if (f.do_amax) {
-      aa.partials = f.partials;
-      aa.npartials = G;
-    }
-    const float s = cta_tensor_scale(aa);
+    __shared__ float s_sh;
+    s = a.static_scale ? *a.static_scale : cta_tensor_scale(a);
     if (tid == 0) s_sh = s;
+    __syncthreads();
+    s = s_sh;
   }
-  __syncthreads();
-  const float s = s_sh;
   if (blockIdx.x == 0 && tid == 0) *a.scale_out = s;
   const float rcp_s = __frcp_rn(s), rcp6 = __frcp_rn(6.0f);
-  if (producer) {
-    for (int q = resident; q < n_c; ++q) {
-      const int sl = first_slot + q, buf = sl % kFusedBufs;
-      const int t = tile_at(q);
-      bool ok = true;
-      if (lane == 0 && sl >= kFusedBufs) {  // the first kFusedBufs slots were issued at the start
-        ok = wait_free(sl);
-        if (ok) issue(sl, t);
+  // decode scale d = E4M3value(byte) * s and -RN(1/d) for every scale byte (0..126)
+  __shared__ float2 dtab[128];
+  for (int i = tid; i < 128; i += NT) {
+    const float dd = __fmul_rn(e4m3_value(static_cast<uint32_t>(i)), s);
+    dtab[i] = make_float2(dd, in_safe_range(dd) ? -__frcp_rn(dd) : 0.0f);
+  }
+  __syncthreads();
+  const int64_t cpitch = a.kpad >> 1;
+  const int nres = a.r >> 4, ntail = (a.kpad - a.K) >> 4;
+
+  for (int m = blockIdx.x; m < mpad; m += gridDim.x) {
+    if (m >= a.M) {  // rows padding the scale layout to a multiple of 128 carry zero scales
+      for (int kb = tid; kb < (a.kpad >> 4); kb += NT) a.sf[sf_offset(m, kb, a.katoms)] = 0;
+      continue;
+    }
+    const __nv_bfloat16* row = a.x + static_cast<int64_t>(m) * a.ldx;
+    uint8_t* crow = a.codes + static_cast<int64_t>(m) * cpitch;
+    // scale byte of (m, kb) at sf_row + (kb / 4) * 512 + kb % 4
+    uint8_t* sf_row = a.sf + static_cast<int64_t>(m >> 7) * a.katoms * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4;
+    double inv = 0.0;
+    if (RMS) inv = a.inv_rms[m];
+    // ---- primary blocks: thread t codes blocks b0 + 128 i + t
+    for (int b0 = 0; b0 < nblk; b0 += NT * kQRowDepth) {
+      uint4 raw[kQRowDepth][2];
+#pragma unroll
+      for (int i = 0; i < kQRowDepth; ++i) {
+        const int b = b0 + NT * i + tid;
+        if (b < nblk) {
+          raw[i][0] = ld_nc_v4(row + 16 * b);
+          raw[i][1] = ld_nc_v4(row + 16 * b + 8);
+        } else {
+          raw[i][0] = raw[i][1] = make_uint4(0, 0, 0, 0);
+        }
       }
-      if (!__shfl_sync(0xFFFFFFFFu, static_cast<int>(ok), 0)) break;
-      build_olist(a, idx_sh, (t % f.tiles_k) * 128, olist[buf], lane);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&full[buf]);
+#pragma unroll
+      for (int i = 0; i < kQRowDepth; ++i) {
+        const int b = b0 + NT * i + tid;
+        if (b0 + NT * i >= nblk) break;  // uniform: no block of this batch position exists
+        const bool valid = b < nblk;
+        const uint32_t w[8] = {raw[i][0].x, raw[i][0].y, raw[i][0].z, raw[i][0].w,
+                               raw[i][1].x, raw[i][1].y, raw[i][1].z, raw[i][1].w};
+        float v[16];
+        float amax;
+        if (RMS) {
+          uint4 g0 = make_uint4(0, 0, 0, 0), g1 = g0;
+          if (valid) {
+            g0 = ld_nc_v4(a.gain + 16 * b);
+            g1 = ld_nc_v4(a.gain + 16 * b + 8);
+          }
+          const uint32_t gs[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            v[2 * j] = rms_apply(bf16_lo(w[j]), inv, bf16_lo(gs[j]));
+            v[2 * j + 1] = rms_apply(bf16_hi(w[j]), inv, bf16_hi(gs[j]));
+          }
+          const float a0 = fmax3_abs(v[0], v[1], v[2]), a1 = fmax3_abs(v[3], v[4], v[5]),
+                      a2 = fmax3_abs(v[6], v[7], v[8]), a3 = fmax3_abs(v[9], v[10], v[11]),
+                      a4 = fmax3_abs(v[12], v[13], v[14]);
+          amax = fmaxf(fmax3(a0, a1, a2), fmax3(a3, a4, fabsf(v[15])));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            v[2 * j] = bf16_lo(w[j]);
+            v[2 * j + 1] = bf16_hi(w[j]);
+          }
+          // |bf16| orders like its bit pattern: the block maximum on packed halves
+          const uint32_t m01 = __vmaxu2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu);
+          const uint32_t m23 = __vmaxu2(w[2] & 0x7FFF7FFFu, w[3] & 0x7FFF7FFFu);
+          const uint32_t m45 = __vmaxu2(w[4] & 0x7FFF7FFFu, w[5] & 0x7FFF7FFFu);
+          const uint32_t m67 = __vmaxu2(w[6] & 0x7FFF7FFFu, w[7] & 0x7FFF7FFFu);
+          const uint32_t mw = __vmaxu2(__vmaxu2(m01, m23), __vmaxu2(m45, m67));
+          amax = __uint_as_float(max(mw & 0xFFFFu, mw >> 16) << 16);
+        }
+        const uint32_t sfv = block_sf(amax, s, rcp_s, rcp6);
+        const float2 dn = dtab[sfv];
+        const float d = dn.x;
+        uint2 cc = make_uint2(0u, 0u);
+        if (d != 0.0f) {
+          uint64_t p[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) p[j] = f2_pack(v[2 * j], v[2 * j + 1]);
+          cc = encode16_nr(p, d, dn.y);
+        }
+        if (valid) *reinterpret_cast<uint2*>(crow + 8 * b) = cc;
+        // a block holding outlier channels keeps its values (bf16: the RMSNorm output is
+        // bf16-rounded), codes and d for the residual step below
+        const int sl = (valid && a.r > 0) ? blk_slot[b] : -1;
+        if (sl >= 0) {
+          uint4* dst = slots + 3 * sl;
+          if (RMS) {
+            dst[0] = make_uint4(pack_bf16x2_rn(v[0], v[1]), pack_bf16x2_rn(v[2], v[3]), pack_bf16x2_rn(v[4], v[5]),
+                                pack_bf16x2_rn(v[6], v[7]));
+            dst[1] = make_uint4(pack_bf16x2_rn(v[8], v[9]), pack_bf16x2_rn(v[10], v[11]),
+                                pack_bf16x2_rn(v[12], v[13]), pack_bf16x2_rn(v[14], v[15]));
+          } else {
+            dst[0] = raw[i][0];
+            dst[1] = raw[i][1];
+          }
+          dst[2] = make_uint4(cc.x, cc.y, __float_as_uint(d), 0u);
+        }
+        // scale bytes: lanes 4i..4i+3 hold blocks b..b+3 (b % 4 == 0 at lane 4i), which sit in
+        // four consecutive bytes of the swizzled layout
+        const uint32_t my = valid ? sfv : 0u;
+        const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, my, 1), s2 = __shfl_down_sync(0xFFFFFFFFu, my, 2),
+                       s3 = __shfl_down_sync(0xFFFFFFFFu, my, 3);
+        if (valid && (lane & 3) == 0) {
+          uint8_t* dst = sf_row + (b >> 2) * 512;
+          if (b + 3 < nblk) {
+            *reinterpret_cast<uint32_t*>(dst) = my | (s1 << 8) | (s2 << 16) | (s3 << 24);
+          } else {
+            dst[0] = static_cast<uint8_t>(my);
+            if (b + 1 < nblk) dst[1] = static_cast<uint8_t>(s1);
+            if (b + 2 < nblk) dst[2] = static_cast<uint8_t>(s2);
+          }
+        }
+      }
     }
-  } else {
-    const int mm = warp * 8 + (lane & 7);
-    const int sf_lane = (mm & 31) * 16 + (mm >> 5) * 4 + (lane >> 3);
-    for (int q = 0; q < n_c; ++q) {
-      const int sl = first_slot + q, buf = sl % kFusedBufs;
-      const int t = tile_at(q);
-      const int tm = t / f.tiles_k, tk = t - tm * f.tiles_k;
-      // resident tiles were waited for in phase 1
-      if (q >= resident &&
-          !mbar_wait(&full[buf], static_cast<uint32_t>((sl / kFusedBufs) & 1), f.wait_ns, &abort_sh))
-        break;
-      code_rows<RMS>(a, xbase + buf * kQTileBytes, tm, tk, s, rcp_s, rcp6, olist[buf], sf_lane);
-      release(sl);
+    if (a.r > 0) {
+      // ---- outlier channels: residual x - E2M1(code) * d (activations) or the value itself
+      // (weights), from the kept blocks
+      __syncthreads();
+      for (int j = tid; j < a.r; j += NT) {
+        const int c = idx_s[j];
+        float res = 0.0f;
+        if (c >= 0) {
+          const uint4* src = slots + 3 * blk_slot[c >> 4];
+          const int e = c & 15;
+          const uint4 vw = src[e >> 3];
+          const int wi = (e >> 1) & 3;
+          const uint32_t word = wi == 0 ? vw.x : wi == 1 ? vw.y : wi == 2 ? vw.z : vw.w;
+          const float xv = (e & 1) ? bf16_hi(word) : bf16_lo(word);
+          res = xv;
+          if (!a.dup) {
+            const uint4 meta = src[2];
+            const uint32_t code = (((e < 8) ? meta.x : meta.y) >> (4 * (e & 7))) & 15u;
+            res = __fsub_rn(xv, __fmul_rn(e2m1_value(code), __uint_as_float(meta.z)));
+          }
+        }
+        stash[j] = res;
+      }
+      __syncthreads();
+    }
+    // ---- appended residual blocks (in idx order, same tensor scale) and zero padding to K_pad
+    for (int rb = tid; rb < ntail; rb += NT) {
+      uint32_t sfv = 0u;
+      uint2 cc = make_uint2(0u, 0u);
+      if (rb < nres) {
+        float v[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = stash[16 * rb + e];
+        const float a0 = fmax3_abs(v[0], v[1], v[2]), a1 = fmax3_abs(v[3], v[4], v[5]),
+                    a2 = fmax3_abs(v[6], v[7], v[8]), a3 = fmax3_abs(v[9], v[10], v[11]),
+                    a4 = fmax3_abs(v[12], v[13], v[14]);
+        sfv = block_sf(fmaxf(fmax3(a0, a1, a2), fmax3(a3, a4, fabsf(v[15]))), s, rcp_s, rcp6);
+        const float2 dn = dtab[sfv];
+        if (dn.x != 0.0f) {
+          uint64_t p[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) p[j] = f2_pack(v[2 * j], v[2 * j + 1]);
+          cc = encode16_nr(p, dn.x, dn.y);
+        }
+      }
+      *reinterpret_cast<uint2*>(crow + ((a.K + 16 * rb) >> 1)) = cc;
+      const int kb = nblk + rb;
+      sf_row[(kb >> 2) * 512 + (kb & 3)] = static_cast<uint8_t>(sfv);
     }
   }
-  __syncthreads();  // both roles are done with the ring
-  if (abort_sh) {
-    if (producer && lane == 0) drain();
-    return;
-  }
-  if (a.kpad == a.K) return;
-  // ---------------------------------------------------------------------- phase 3: tail
-  if (!grid_barrier(f.flags + 32 + G, f.flags + 16, G, f.epoch + 1, f.wait_ns, &abort_sh)) return;
-  tail_items(a, f.mpad, s, rcp_s, rcp6);
 }
 
 }  // namespace arc

@@ -42,7 +42,7 @@ def test_size_queries(L):
         assert L.arc_kpad(kaug) == kp == O.kpad(kaug)
         assert L.arc_nvfp4_codes_bytes(rows, kaug) == rows * kp // 2
         assert L.arc_nvfp4_sf_bytes(rows, kaug) == O.sf_swizzled_bytes(rows, kp // 16)
-    assert L.arc_quantize_workspace_bytes(4096, 128) >= 4 + 4096 * 128 * 4 + 4096 * 8
+    assert L.arc_quantize_workspace_bytes(4096, 128) >= 4 + 4096 * 8  # partials, 1/rms per row
     assert L.arc_status_str(5) == b"ARC_ERR_TIMEOUT"
 
 
