@@ -27,8 +27,9 @@
 //                every quarter q, column base + n/32). Register stores keep the tensor pipe free
 //                for MMAs; tcgen05.cp of the same bytes costs the pipe ~70 cycles per copy.
 //   warps 7..14  epilogue: tcgen05.ld of the fp32 accumulator (warp w owns TMEM lane quarter
-//                w%4 = tile rows 32*(w%4)..+31, and one 128-column half), scale by alpha,
-//                optional residual add, bf16 stores.
+//                w%4 = tile rows 32*(w%4)..+31, and one 128-column half), scale by alpha; bf16
+//                output staged 32 x 16 at a time in shared memory and written by TMA stores (the
+//                residual-add form reads the add term and stores directly).
 // TMEM (512 columns): fp32 accumulator 128 lanes x 256 columns (two of them for bf16); fp4
 // keeps one and uses columns 256..511 as four 64-column scale sets, one per pipeline stage
 // (B scales at +0..31, 8 columns per K=64 step; A scales at +32 + 4k + quarter).
@@ -66,10 +67,24 @@ struct GemmTraits<false> {
   static constexpr int SF_COL0 = 0, SF_SET_COLS = 0;
 };
 
+// Output staging for the TMA-store epilogue: per epilogue warp one 32-row x 16-column bf16 chunk.
+constexpr int kEpiStageBytes = 32 * 16 * 2;
+
 template <bool FP4>
 constexpr int gemm_smem_bytes() {
-  return GemmTraits<FP4>::STAGES * GemmTraits<FP4>::STAGE_BYTES + 1024 + 256;
+  return GemmTraits<FP4>::STAGES * GemmTraits<FP4>::STAGE_BYTES + 8 * kEpiStageBytes + 1024 + 256;
 }
+
+// TMA tensor store of a box from shared memory (bulk-group completion), and its waits.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(m),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 struct GemmArgs {
   int M, N;
@@ -136,11 +151,13 @@ constexpr int kGemmEpiWarp0 = 7;
 
 template <bool FP4, bool ADD>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
+    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+           const __grid_constant__ CUtensorMap tmY, const GemmArgs g) {
   using T = GemmTraits<FP4>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + T::STAGES * T::STAGE_BYTES);
+  uint8_t* staging = smem + T::STAGES * T::STAGE_BYTES;  // 8 x 1 KB, one per epilogue warp
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + 8 * kEpiStageBytes);
   uint64_t* empty = full + T::STAGES;
   uint64_t* ready = empty + T::STAGES;  // fp4: the stage's scales are in TMEM
   uint64_t* acc_full = ready + T::STAGES;
@@ -168,6 +185,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (!ADD) tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, T::TMEM_COLS);
@@ -400,14 +418,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[acc]);
-        if (row_ok) {
+        // stores through the warp's staging chunk: thread i writes row i's 16 columns, one TMA
+        // store moves the 32 x 16 box to Y (clipped at the matrix edges)
+        uint8_t* stg = staging + (warp - kGemmEpiWarp0) * kEpiStageBytes;
+        const int row0 = tm * T::BM + q * 32;
 #pragma unroll
-          for (int j = 0; j < HB / 8; ++j) {
-            const int col = col0 + 8 * j;
-            if (col < g.N)
-              *reinterpret_cast<uint4*>(yrow + col) = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        for (int c = 0; c < HB / 16; ++c) {
+          uint4* dst = reinterpret_cast<uint4*>(stg + lane * 32);
+          dst[0] = make_uint4(pk[8 * c], pk[8 * c + 1], pk[8 * c + 2], pk[8 * c + 3]);
+          dst[1] = make_uint4(pk[8 * c + 4], pk[8 * c + 5], pk[8 * c + 6], pk[8 * c + 7]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmY, stg, col0 + 16 * c, row0);
+            bulk_commit_group();
+            bulk_wait_read_all();  // the chunk may be overwritten once the TMA has read it
           }
+          __syncwarp();
         }
+        (void)row_ok;
+        (void)yrow;
       } else {
 #pragma unroll
         for (int c = 0; c < HB / 32; ++c) {
@@ -446,6 +476,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         acc_phase ^= 1u;
       }
     }
+    if (!ADD && lane == 0) bulk_wait_all();  // every output store has completed
   }
   __syncthreads();
   if (warp == 1) {

@@ -103,6 +103,20 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Y [outer, inner] bf16, row pitch in bytes, as the target of 32-row x 16-column TMA stores
+// (no swizzle; the staging chunk is 32 rows of 32 bytes).
+bool make_store_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch_bytes) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {16, 32};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int take_inject() {
   std::lock_guard<std::mutex> lk(g_mu);
   const int k = g_inject;
@@ -221,10 +235,15 @@ arc_status gemm_launch(const CUtensorMap& ta, const CUtensorMap& tb, GemmArgs g,
   const int ntiles = g.tiles_m * g.tiles_n;
   const unsigned grid = static_cast<unsigned>(std::min(ntiles, sms));
   const int smem = arc::gemm_smem_bytes<FP4>();
+  CUtensorMap ty;
+  std::memset(&ty, 0, sizeof(ty));
+  if (!add && !make_store_map(&ty, g.y, static_cast<uint64_t>(g.N), static_cast<uint64_t>(g.M),
+                              static_cast<uint64_t>(g.ldy) * 2))
+    return ARC_ERR_CUDA;
   if (add)
-    arc::k_gemm<FP4, true><<<grid, arc::kGemmThreads, smem, s>>>(ta, tb, g);
+    arc::k_gemm<FP4, true><<<grid, arc::kGemmThreads, smem, s>>>(ta, tb, ty, g);
   else
-    arc::k_gemm<FP4, false><<<grid, arc::kGemmThreads, smem, s>>>(ta, tb, g);
+    arc::k_gemm<FP4, false><<<grid, arc::kGemmThreads, smem, s>>>(ta, tb, ty, g);
   return launch_status();
 }
 
