@@ -1,14 +1,25 @@
 #!/usr/bin/env python
 """Benchmark of the NVFP4 + augmented-residual-channel prefill path on B200.
 
-One step = the Llama-3-8B-shaped prefill projections on one token batch of M = 4096:
-for each of qkv (K=4096, N=6144), o (4096, 4096), gateup (4096, 28672), down (14336, 4096):
-  dynamic-scale activation quantization with r = 128 residual channels (abs-max pass, fused
-  quantize + residual stash, residual tail) -> block-scaled NVFP4 GEMM of depth K + r -> bf16 Y.
-Weights are packed and outlier channels calibrated once, before timing (offline steps).
+Default workload (the headline): the Llama-3-8B-shaped prefill projections on one token batch of
+M = 4096. One step = for each of qkv (K=4096, N=6144), o (4096, 4096), gateup (4096, 28672),
+down (14336, 4096): dynamic-scale activation quantization with r = 128 residual channels
+(abs-max pass, then the coding pass with the residual blocks) -> block-scaled NVFP4 GEMM of
+depth K + r -> bf16 Y. Weights are packed and outlier channels calibrated once, before timing
+(offline steps).
+
+Other workloads (--workload), same timing rules:
+  mlp70b     M = 16384: gate|up 8192 -> 57344, down 28672 -> 8192, r = 256
+  stress     M = 2048, K = N = 4096, Student-t(3) activations, outlier fraction {0, 0.1, 1, 5} %
+             x r in {0, 32, 128, 256}; also the relative error of each output against the BF16
+             product (the library's own BF16 GEMM of the same inputs)
+  recurrent  the shared 2-sublayer SwiGLU block (d = 2048, ffn = 8192, RMSNorm, residual add)
+             applied T = 16 times to H [4096, 2048]: one prefill per k_low in {0, 8, 12, 16}
+             (steps before k_low in NVFP4 + ARC with r = 64, the rest BF16); time per prefill,
+             speedup against k_low = 0 and the hidden-state error against all-BF16
 
 Metric: NVFP4 ARC GEMM TFLOP/s = sum over the step of 2*M*N*(K+r) / step time, with the fused
-activation quantizer's GB/s (read X + write codes + scale bytes) reported beside it.
+activation quantizer's GB/s (read X + write codes + scale bytes) beside it.
 Timing: CUDA events on the launching stream around every step and every kernel call; the L2 is
 flushed (a 256 MiB write) before every timed step, outside the events. Multi-GPU: one process
 per GPU, each rank runs the same step on its own token batch (weak scaling, no data-path
@@ -33,25 +44,65 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-PROJ = [("qkv", 4096, 6144), ("o", 4096, 4096), ("gateup", 4096, 28672), ("down", 14336, 4096)]
-M_TOKENS = 4096
-R = 128
 METRIC = "NVFP4 ARC GEMM TFLOP/s (% FP4 peak) + fused act-quant GB/s, 1×B200"
 UNIT = "TFLOP/s"
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLOP/s)
 
 
-def step_flops(M=M_TOKENS):
-    return sum(2.0 * M * N * (K + R) for _, K, N in PROJ)
+# ---------------------------------------------------------------------------------------------
+# Workloads: lists of linear layers (name, M, K, N, r, generator)
+# ---------------------------------------------------------------------------------------------
+
+def layer_set(workload: str):
+    import workloads as W
+
+    out = []
+    if workload == "llama8b":
+        M = W.LLAMA8B_M
+        for name, (_, K, N) in W.LLAMA8B_PROJ.items():
+            out.append(dict(name=name, M=M, K=K, N=N, r=W.LLAMA8B_R,
+                            gen=lambda rows, row0, name=name: W.llama8b(name, rows=rows, row0=row0)))
+        desc = f"llama8b-prefill-projections: M={M} tokens, qkv/o/gateup/down, r={W.LLAMA8B_R}"
+    elif workload == "mlp70b":
+        M = W.MLP70B_M
+        for name, (_, K, N) in W.MLP70B_PROJ.items():
+            out.append(dict(name=name, M=M, K=K, N=N, r=W.MLP70B_R,
+                            gen=lambda rows, row0, name=name: W.mlp70b(name, rows=rows, row0=row0)))
+        desc = f"mlp70b-prefill: M={M} tokens, gateup 8192->57344, down 28672->8192, r={W.MLP70B_R}"
+    elif workload == "stress":
+        c = W.STRESS
+        cache = {}
+
+        def gen(rows, row0, frac):
+            key = (frac, rows, row0)
+            if key not in cache:
+                cache.clear()
+                cache[key] = W.stress(frac, rows=rows)
+            return cache[key]
+
+        for frac in c["fracs"]:
+            for r in c["rs"]:
+                out.append(dict(name=f"frac{frac:g}-r{r}", M=c["M"], K=c["K"], N=c["N"], r=r,
+                                gen=lambda rows, row0, frac=frac: gen(rows, row0, frac)))
+        desc = (f"outlier-stress sweep: M={c['M']}, K=N={c['K']}, Student-t(3), outlier fraction "
+                f"{list(c['fracs'])} x r {list(c['rs'])}")
+    else:
+        raise ValueError(workload)
+    return out, desc
 
 
-def quant_bytes(M=M_TOKENS):
+def kpad(k):
+    return (k + 63) // 64 * 64
+
+
+def layer_flops(L):
+    return 2.0 * L["M"] * L["N"] * (L["K"] + L["r"])
+
+
+def layer_quant_bytes(L):
     """Algorithmic bytes of the quantizer: read X once, write codes and scale bytes."""
-    tot = 0
-    for _, K, _ in PROJ:
-        kp = (K + R + 63) // 64 * 64
-        tot += 2 * M * K + M * kp // 2 + M * kp // 16
-    return tot
+    kp = kpad(L["K"] + L["r"])
+    return 2 * L["M"] * L["K"] + L["M"] * kp // 2 + L["M"] * kp // 16
 
 
 def peaks():
@@ -147,44 +198,50 @@ class ClockSampler:
                 "source": "nvml"}
 
 
+def _ev():
+    return torch.cuda.Event(enable_timing=True)
+
+
+def _barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
 # ---------------------------------------------------------------------------------------------
-# Our arm
+# Our arm: linear-layer workloads
 # ---------------------------------------------------------------------------------------------
 
-def make_inputs(rank: int, device):
+def run_layers(args, rank, world, device, layers, with_error=False):
+    import nvfp4_block_scaled_arc_b200 as arc
     import workloads as W
 
-    xs, ws = {}, {}
-    for name, K, N in PROJ:
-        d = W.llama8b(name, rows=M_TOKENS, row0=rank * M_TOKENS)
-        xs[name] = W.to_torch_bf16(d["x"])
-        ws[name] = W.to_torch_bf16(d["w"]).to(device)
-    return xs, ws
-
-
-def run_ours(args, rank, world, device):
-    import nvfp4_block_scaled_arc_b200 as arc
-
     stream = torch.cuda.Stream(device=device)
-    xs_host, ws = make_inputs(rank, device)
+    xs_host, xs, idx, packed, qa, ys, wsp, errs = {}, {}, {}, {}, {}, {}, {}, {}
     with torch.cuda.stream(stream):
-        xs = {k: v.to(device, non_blocking=False) for k, v in xs_host.items()}
-        idx, packed, qa, ys, wsp = {}, {}, {}, {}, {}
-        for name, K, N in PROJ:
-            idx[name] = arc.calibrate_outliers(xs[name], R, stream=stream)
-            packed[name] = arc.pack_weight_nvfp4(ws[name], idx[name], stream=stream)
+        for L in layers:
+            name, M, r = L["name"], L["M"], L["r"]
+            d = L["gen"](M, rank * M)
+            xs_host[name] = W.to_torch_bf16(d["x"])
+            xs[name] = xs_host[name].to(device)
+            w = W.to_torch_bf16(d["w"]).to(device)
+            idx[name] = arc.calibrate_outliers(xs[name], r, stream=stream) if r else None
+            packed[name] = arc.pack_weight_nvfp4(w, idx[name], stream=stream)
             qa[name] = arc.quantize_act_nvfp4(xs[name], idx[name], stream=stream)
-            ys[name] = torch.empty(M_TOKENS, N, dtype=torch.bfloat16, device=device)
-            wsp[name] = torch.empty(arc.quantize_workspace_bytes(M_TOKENS, R), dtype=torch.uint8, device=device)
+            ys[name] = torch.empty(M, L["N"], dtype=torch.bfloat16, device=device)
+            wsp[name] = torch.empty(arc.quantize_workspace_bytes(M, r), dtype=torch.uint8, device=device)
+            if with_error:
+                # relative error of the NVFP4 + ARC output against the BF16 product of the inputs
+                y = arc.gemm_nvfp4(qa[name], packed[name], stream=stream).float()
+                yb = arc.gemm_bf16(xs[name], w, stream=stream).float()
+                errs[name] = (torch.linalg.norm(y - yb) / torch.linalg.norm(yb)).item()
+            del w
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
     stream.synchronize()
-    del ws
-
-    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
 
     def step(rec):
-        for name, K, N in PROJ:
-            e0, e1, e2 = (ev(), ev(), ev()) if rec is not None else (None, None, None)
+        for L in layers:
+            name = L["name"]
+            e0, e1, e2 = (_ev(), _ev(), _ev()) if rec is not None else (None, None, None)
             if e0 is not None:
                 e0.record(stream)
             arc.quantize_act_nvfp4(xs[name], idx[name], out=qa[name], workspace=wsp[name], stream=stream)
@@ -195,7 +252,6 @@ def run_ours(args, rank, world, device):
                 e2.record(stream)
                 rec.append((e0, e1, e2))
 
-    # warm-up
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             flush.zero_()
@@ -204,18 +260,14 @@ def run_ours(args, rank, world, device):
     if arc.last_device_status(stream) != 0:
         raise RuntimeError("device status set during warm-up")
 
-    def barrier():
-        if world > 1:
-            torch.distributed.barrier()
-
     step_ev, kern = [], []
-    barrier()
+    _barrier(world)
     torch.cuda.synchronize(device)
     with ClockSampler(device) as clk:
         with torch.cuda.stream(stream):
             for _ in range(args.steps):
                 flush.zero_()
-                s0, s1 = ev(), ev()
+                s0, s1 = _ev(), _ev()
                 s0.record(stream)
                 rec = []
                 step(rec)
@@ -223,138 +275,269 @@ def run_ours(args, rank, world, device):
                 step_ev.append((s0, s1))
                 kern.append(rec)
         torch.cuda.synchronize(device)
-    barrier()
+    _barrier(world)
     if arc.last_device_status(stream) != 0:
         raise RuntimeError("device status set during the timed steps")
-    step_ms = [a.elapsed_time(b) for a, b in step_ev]
-    total_ms = sum(step_ms)
+    total_ms = sum(a.elapsed_time(b) for a, b in step_ev)
     q_ms = sum(r[0].elapsed_time(r[1]) for rec in kern for r in rec)
     g_ms = sum(r[1].elapsed_time(r[2]) for rec in kern for r in rec)
-    per_proj = {}
-    for i, (name, K, N) in enumerate(PROJ):
-        gq = [rec[i][0].elapsed_time(rec[i][1]) for rec in kern]
-        gg = [rec[i][1].elapsed_time(rec[i][2]) for rec in kern]
-        kp = (K + R + 63) // 64 * 64
-        per_proj[name] = {
-            "quant_us": 1e3 * statistics.mean(gq),
-            "quant_gbs": (2 * M_TOKENS * K + M_TOKENS * kp // 2 + M_TOKENS * kp // 16) / (statistics.mean(gq) * 1e-3) / 1e9,
-            "gemm_us": 1e3 * statistics.mean(gg),
-            "gemm_tflops": 2.0 * M_TOKENS * N * (K + R) / (statistics.mean(gg) * 1e-3) / 1e12,
-        }
+    per_layer = {}
+    for i, L in enumerate(layers):
+        gq = statistics.mean(rec[i][0].elapsed_time(rec[i][1]) for rec in kern)
+        gg = statistics.mean(rec[i][1].elapsed_time(rec[i][2]) for rec in kern)
+        per_layer[L["name"]] = {"quant_us": 1e3 * gq, "quant_gbs": layer_quant_bytes(L) / (gq * 1e-3) / 1e9,
+                                "gemm_us": 1e3 * gg, "gemm_tflops": layer_flops(L) / (gg * 1e-3) / 1e12}
+        if with_error:
+            per_layer[L["name"]]["rel_err_vs_bf16"] = errs[L["name"]]
     clocks = clk.summary()
 
     # e2e through the public API with host buffers: pinned X in, Y out, every step
-    xs_pin = {k: v.pin_memory() for k, v in xs_host.items()}
-    ys_pin = {name: torch.empty(M_TOKENS, N, dtype=torch.bfloat16).pin_memory() for name, _, N in PROJ}
-    h2d = sum(v.numel() * 2 for v in xs_pin.values())
-    d2h = sum(v.numel() * 2 for v in ys_pin.values())
-
-    def e2e_step():
-        for name, K, N in PROJ:
-            xs[name].copy_(xs_pin[name], non_blocking=True)
-            arc.quantize_act_nvfp4(xs[name], idx[name], out=qa[name], workspace=wsp[name], stream=stream)
-            arc.gemm_nvfp4(qa[name], packed[name], out=ys[name], stream=stream)
-            ys_pin[name].copy_(ys[name], non_blocking=True)
-
-    e2e_ms = float("nan")
+    e2e_ms, h2d, d2h = float("nan"), 0, 0
     if not args.no_e2e:
+        xs_pin = {k: v.pin_memory() for k, v in xs_host.items()}
+        ys_pin = {L["name"]: torch.empty(L["M"], L["N"], dtype=torch.bfloat16).pin_memory() for L in layers}
+        h2d = sum(v.numel() * 2 for v in xs_pin.values())
+        d2h = sum(v.numel() * 2 for v in ys_pin.values())
+
+        def e2e_step():
+            for L in layers:
+                name = L["name"]
+                xs[name].copy_(xs_pin[name], non_blocking=True)
+                arc.quantize_act_nvfp4(xs[name], idx[name], out=qa[name], workspace=wsp[name], stream=stream)
+                arc.gemm_nvfp4(qa[name], packed[name], out=ys[name], stream=stream)
+                ys_pin[name].copy_(ys[name], non_blocking=True)
+
         with torch.cuda.stream(stream):
             for _ in range(max(1, min(args.warmup, 2))):
                 e2e_step()
         stream.synchronize()
-        barrier()
+        _barrier(world)
         e2e_ev = []
         with torch.cuda.stream(stream):
             for _ in range(args.steps):
-                a, b = ev(), ev()
+                a, b = _ev(), _ev()
                 a.record(stream)
                 e2e_step()
                 b.record(stream)
                 e2e_ev.append((a, b))
         stream.synchronize()
-        barrier()
+        _barrier(world)
         e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
 
     t = torch.tensor([total_ms, q_ms, g_ms, e2e_ms], dtype=torch.float64, device=device)
     if world > 1:
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     total_ms, q_ms, g_ms, e2e_ms = t.tolist()
-    return dict(total_ms=total_ms, q_ms=q_ms, g_ms=g_ms, e2e_ms=e2e_ms, per_proj=per_proj, clocks=clocks,
-                h2d=h2d, d2h=d2h, launches=args.steps * len(PROJ) * 2)
+    return dict(total_ms=total_ms, q_ms=q_ms, g_ms=g_ms, e2e_ms=e2e_ms, per_layer=per_layer, clocks=clocks,
+                h2d=h2d, d2h=d2h, launches=args.steps * len(layers) * 3)
+
+
+def layers_line(args, world, layers, desc, res):
+    pk, src = peaks()
+    step_flops = sum(layer_flops(L) for L in layers)
+    qbytes = sum(layer_quant_bytes(L) for L in layers)
+    value = step_flops * world * args.steps / (res["total_ms"] * 1e-3) / 1e12
+    achieved = step_flops * args.steps / (res["g_ms"] * 1e-3) / 1e12
+    quant_gbs = qbytes * args.steps / (res["q_ms"] * 1e-3) / 1e9
+    peak = pk["bf16_tflops"] * FP4_OVER_BF16
+    return {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": res["total_ms"] / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e2m1 x e2m1 -> f32 (bf16 out)",
+        "data": "synthetic (seeded; random weights and activations of the stated shapes)",
+        "config": {"workload": desc, "l2": "flushed (256 MiB write) before every step",
+                   "parallelism": f"replicas x{world}"},
+        "quant_gbs": quant_gbs,
+        "gemm_only_tflops": achieved,
+        "pct_fp4_peak": 100.0 * value / peak,
+        "per_projection": res["per_layer"],
+        "roofline": {"bound": "tensor", "kernel": f"k_gemm<nvfp4> (all {len(layers)} launches of a step)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{src} bf16 burst {pk['bf16_tflops']} TFLOP/s x {FP4_OVER_BF16:g} "
+                                    f"(nominal FP4/BF16 dense ratio)",
+                     "traffic": ncu_traffic() if args.workload == "llama8b" else None},
+        "quant_roofline": {"bound": "hbm", "kernel": "k_amax + k_quant_rows", "achieved": quant_gbs,
+                           "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": quant_gbs / pk["hbm_gbs"],
+                           "peak_source": f"{src} copy bandwidth"},
+        "clocks": res["clocks"],
+        "e2e": None if args.no_e2e else {
+            "value": step_flops * world * args.steps / (res["e2e_ms"] * 1e-3) / 1e12, "unit": UNIT,
+            "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
+        "gpu_launches": res["launches"],
+    }
+
+
+# ---------------------------------------------------------------------------------------------
+# Our arm: the RAMP-style recurrent prefill
+# ---------------------------------------------------------------------------------------------
+
+def run_recurrent(args, rank, world, device):
+    import nvfp4_block_scaled_arc_b200 as arc
+    import workloads as W
+
+    c = W.RECURRENT
+    S, d, F, T, r, eps = c["S"], c["d"], c["ffn"], c["T"], c["r"], c["eps"]
+    rec = W.recurrent()
+    stream = torch.cuda.Stream(device=device)
+    with torch.cuda.stream(stream):
+        h0 = W.to_torch_bf16(rec["h"]).to(device)
+        subs = []
+        for L in rec["layers"]:
+            wgu, wd, gain = (W.to_torch_bf16(L[k]).to(device) for k in ("wgu", "wd", "gain"))
+            # offline calibration on a BF16 pass of the block's first step
+            n = arc.rmsnorm_bf16(h0, gain, eps, stream=stream)
+            idx_gu = arc.calibrate_outliers(n, r, stream=stream)
+            act = arc.silu_mul_bf16(arc.gemm_bf16(n, wgu, stream=stream), stream=stream)
+            idx_d = arc.calibrate_outliers(act, r, stream=stream)
+            subs.append(dict(gain=gain, wgu=wgu, wd=wd, idx_gu=idx_gu, idx_d=idx_d,
+                             gu_q=arc.pack_weight_nvfp4(wgu, idx_gu, stream=stream),
+                             d_q=arc.pack_weight_nvfp4(wd, idx_d, stream=stream)))
+        blk = arc.RecurrentBlock(d, F, eps, subs)
+        wsp = torch.empty(blk.workspace_bytes(S), dtype=torch.uint8, device=device)
+        h = torch.empty_like(h0)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    stream.synchronize()
+    k_lows = list(c["k_lows"])
+    # GEMM flops of one prefill (both sublayers, every step): gate|up and down; NVFP4 steps run
+    # depth K + r
+    f_bf16 = 2 * (2.0 * S * (2 * F * d + d * F))
+    f_fp4 = 2 * (2.0 * S * (2 * F * (d + r) + d * (F + r)))
+
+    def prefill(k):
+        h.copy_(h0)
+        arc.recurrent_prefill(h, blk, T, k, workspace=wsp, stream=stream)
+
+    out = {}
+    with torch.cuda.stream(stream):
+        for k in k_lows:
+            prefill(k)
+            out[k] = h.float().clone()
+    stream.synchronize()
+    ref = out[0]
+    fidelity = {k: (torch.linalg.norm(out[k] - ref) / torch.linalg.norm(ref)).item() for k in k_lows}
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            for k in k_lows:
+                flush.zero_()
+                prefill(k)
+    stream.synchronize()
+    times = {k: [] for k in k_lows}
+    _barrier(world)
+    torch.cuda.synchronize(device)
+    evs = []
+    with ClockSampler(device) as clk:
+        with torch.cuda.stream(stream):
+            for _ in range(args.steps):
+                for k in k_lows:
+                    flush.zero_()
+                    a, b = _ev(), _ev()
+                    a.record(stream)
+                    prefill(k)
+                    b.record(stream)
+                    evs.append((k, a, b))
+        torch.cuda.synchronize(device)
+    _barrier(world)
+    if arc.last_device_status(stream) != 0:
+        raise RuntimeError("device status set during the timed prefills")
+    for k, a, b in evs:
+        times[k].append(a.elapsed_time(b))
+    t = torch.tensor([statistics.mean(times[k]) for k in k_lows], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms = dict(zip(k_lows, t.tolist()))
+    per = {}
+    for k in k_lows:
+        fl = (k * f_fp4 + (T - k) * f_bf16) * world
+        per[f"k_low={k}"] = {"ms": ms[k], "speedup_vs_all_bf16": ms[k_lows[0]] / ms[k],
+                             "gemm_tflops": fl / (ms[k] * 1e-3) / 1e12,
+                             "hidden_state_rel_err_vs_all_bf16": fidelity[k]}
+    kk = 12 if 12 in ms else k_lows[-1]
+    # kernels per prefill: NVFP4 step = 2 x (2 quantizer launches + GEMM + SiLU + 2 quantizer
+    # launches + GEMM), BF16 step = 2 x (RMSNorm + GEMM + SiLU + GEMM)
+    launches = args.steps * sum(k * 2 * 7 + (T - k) * 2 * 4 for k in k_lows)
+    return {
+        "metric": f"RAMP-style recurrent prefill time (T={T}, first {kk} steps NVFP4+ARC then BF16), 1×B200",
+        "value": ms[kk], "unit": "ms", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sum(ms.values()), "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e2m1 x e2m1 -> f32 (NVFP4 steps), bf16 x bf16 -> f32 (BF16 steps); bf16 hidden state",
+        "data": "synthetic (seeded; random weights and hidden state of the stated shapes)",
+        "config": {"workload": f"recurrent SwiGLU block: S={S}, d={d}, ffn={F}, 2 pre-norm sublayers, T={T}, "
+                               f"k_low in {k_lows}, r={r}",
+                   "l2": "flushed (256 MiB write) before every prefill", "parallelism": f"replicas x{world}"},
+        "per_k_low": per, "clocks": clk.summary(), "e2e": None, "gpu_launches": launches,
+    }
 
 
 # ---------------------------------------------------------------------------------------------
 # Oracle arm (CPU)
 # ---------------------------------------------------------------------------------------------
 
-def oracle_sample_step(rows: int, cache: dict):
-    """One bounded sample of the step on the CPU oracle: `rows` token rows of every projection
-    through calibration-free quantization (idx from the full-batch calibration cached up
-    front), and the FP64 GEMM of those rows against all N outputs. Returns algorithmic flops."""
+def oracle_cache(layers, n_rows: int):
     import oracle as O
-
-    flops = 0.0
-    for name, K, N in PROJ:
-        c = cache[name]
-        x = c["x"][:rows]
-        ac, asf = O.quantize_act(x, c["idx"], c["sa"])
-        O.gemm_nvfp4_f64(ac, asf, c["sa"], c["bc"], c["bsf"], c["sw"])
-        flops += 2.0 * rows * N * (K + R)
-    return flops
-
-
-def oracle_cache(n_rows: int):
-    import oracle as O
-    import workloads as W
 
     cache = {}
-    for name, K, N in PROJ:
-        d = W.llama8b(name, rows=n_rows)
-        idx = O.calibrate(d["x"], R)
-        sa = O.tensor_scale(O.amax(d["x"]))
+    for L in layers:
+        d = L["gen"](n_rows, 0)
+        x = d["x"][:n_rows]
+        idx = O.calibrate(x, L["r"]) if L["r"] else np.zeros(0, np.int32)
+        sa = O.tensor_scale(O.amax(x))
         sw = O.tensor_scale(O.amax(d["w"]))
-        bc, bsf = O.pack_weight(d["w"], idx, sw)
-        cache[name] = dict(x=d["x"], idx=idx, sa=sa, sw=sw, bc=bc, bsf=bsf)
+        bc, bsf = O.pack_weight(d["w"], idx, sw)  # every output column needs the full weight
+        cache[L["name"]] = dict(x=x, idx=idx, sa=sa, sw=sw, bc=bc, bsf=bsf)
     return cache
 
 
-def cpu_baseline(rows: int | None = None):
+def oracle_sample_step(layers, rows: int, cache: dict):
+    """One bounded sample of the step on the CPU oracle: `rows` token rows of every layer through
+    quantization (idx from the sample's calibration, cached up front) and the FP64 GEMM of those
+    rows against all N outputs. Returns algorithmic flops."""
+    import oracle as O
+
+    flops = 0.0
+    for L in layers:
+        c = cache[L["name"]]
+        ac, asf = O.quantize_act(c["x"][:rows], c["idx"], c["sa"])
+        O.gemm_nvfp4_f64(ac, asf, c["sa"], c["bc"], c["bsf"], c["sw"])
+        flops += 2.0 * rows * L["N"] * (L["K"] + L["r"])
+    return flops
+
+
+def cpu_baseline(layers, rows: int | None = None):
     """The oracle on the host cores: `rows` token rows (default two per host thread, so every
-    thread works) of each projection, about 10-30 s of CPU work."""
+    thread works) of each layer, about 10-30 s of CPU work."""
     import oracle as O
 
     rows = rows or 2 * O._threads()
-    cache = oracle_cache(max(rows, 64))
+    cache = oracle_cache(layers, max(rows, 64))
     t0 = time.perf_counter()
-    flops = oracle_sample_step(rows, cache)
+    flops = oracle_sample_step(layers, rows, cache)
     dt = time.perf_counter() - t0
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": min(O._threads(), rows), "kind": "oracle",
-            "sample": f"{rows} token row(s) of each of the 4 projections (quantize + FP64 GEMM against all N), "
-                      f"{dt:.1f} s"}
+            "sample": f"{rows} token row(s) of each of the {len(layers)} layers (quantize + FP64 GEMM against "
+                      f"all N), {dt:.1f} s"}
 
 
-def run_reference(args, rank, world):
+def run_reference(args, rank, world, layers, desc):
     if rank != 0:
         return
     import oracle as O
 
     rows = O._threads()  # one token row per host thread per step
-    cache = oracle_cache(max(rows, 64))
+    cache = oracle_cache(layers, max(rows, 64))
     for _ in range(args.warmup):
-        oracle_sample_step(rows, cache)
+        oracle_sample_step(layers, rows, cache)
     t0 = time.perf_counter()
     flops = 0.0
     for _ in range(args.steps):
-        flops += oracle_sample_step(rows, cache)
+        flops += oracle_sample_step(layers, rows, cache)
     dt = time.perf_counter() - t0
     v = flops / dt / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "llama8b-prefill-projections M=4096 r=128 (oracle on a row sample)",
-                       "sample_rows_per_projection": rows},
+            "config": {"workload": f"{desc} (oracle on a row sample)", "sample_rows_per_projection": rows},
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": O._threads(), "kind": "oracle",
-                             "sample": f"{rows} token rows of each of the 4 projections per step "
+                             "sample": f"{rows} token rows of each of the {len(layers)} layers per step "
                                        f"(quantize + FP64 GEMM against all N)"},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -368,23 +551,31 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama8b", choices=["llama8b", "mlp70b", "stress", "recurrent"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
-    ap.add_argument("--proj", default="all", help="profiling: run only this projection (qkv, o, gateup, down)")
+    ap.add_argument("--proj", default="all", help="profiling: run only this layer (e.g. qkv, gateup)")
     args = ap.parse_args()
-    if args.proj != "all":
-        global PROJ
-        PROJ = [p for p in PROJ if p[0] == args.proj]
-        if not PROJ:
-            ap.error("unknown --proj")
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    layers, desc = None, None
+    if args.workload != "recurrent":
+        layers, desc = layer_set(args.workload)
+        if args.proj != "all":
+            layers = [L for L in layers if L["name"] == args.proj]
+            if not layers:
+                ap.error("unknown --proj")
     if args.impl == "reference":
-        run_reference(args, rank, world)
+        if layers is None:
+            if rank == 0:
+                print(json.dumps({"impl": "reference",
+                                  "unavailable": "the oracle arm times the linear-layer workloads only"}))
+            return
+        run_reference(args, rank, world, layers, desc)
         return
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
@@ -393,44 +584,14 @@ def main():
 
         torch.distributed.init_process_group("nccl", device_id=device, timeout=datetime.timedelta(seconds=180))
     try:
-        res = run_ours(args, rank, world, device)
+        if args.workload == "recurrent":
+            line = run_recurrent(args, rank, world, device)
+        else:
+            res = run_layers(args, rank, world, device, layers, with_error=args.workload == "stress")
+            line = layers_line(args, world, layers, desc, res) if rank == 0 else None
+            if rank == 0 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline(layers)
         if rank == 0:
-            pk, src = peaks()
-            flops = step_flops() * world
-            value = flops * args.steps / (res["total_ms"] * 1e-3) / 1e12
-            gemm_flops_launch = step_flops()  # all GEMM launches of a step (one rank)
-            g_avg_s = res["g_ms"] * 1e-3 / args.steps
-            achieved = gemm_flops_launch / g_avg_s / 1e12
-            peak = pk["bf16_tflops"] * FP4_OVER_BF16
-            traffic = ncu_traffic()
-            line = {
-                "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": res["total_ms"] / args.steps, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "e2m1 x e2m1 -> f32 (bf16 out)",
-                "data": "synthetic (seeded; random weights and activations of the stated shapes)",
-                "config": {"workload": "llama8b-prefill-projections: M=4096 tokens, qkv/o/gateup/down, r=128",
-                           "tokens_per_gpu": M_TOKENS, "r": R, "l2": "flushed (256 MiB write) before every step",
-                           "parallelism": f"replicas x{world}"},
-                "quant_gbs": quant_bytes() * args.steps / (res["q_ms"] * 1e-3) / 1e9,
-                "gemm_only_tflops": achieved,
-                "pct_fp4_peak": 100.0 * value / peak,
-                "per_projection": res["per_proj"],
-                "roofline": {"bound": "tensor", "kernel": "k_gemm<nvfp4> (all 4 launches of a step)",
-                             "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                             "peak_source": f"{src} bf16 burst {pk['bf16_tflops']} TFLOP/s x {FP4_OVER_BF16:g} "
-                                            f"(nominal FP4/BF16 dense ratio)",
-                             "traffic": traffic},
-                "quant_roofline": {"bound": "hbm", "achieved": quant_bytes() * args.steps / (res["q_ms"] * 1e-3) / 1e9,
-                                   "peak": pk["hbm_gbs"], "unit": "GB/s",
-                                   "frac": quant_bytes() * args.steps / (res["q_ms"] * 1e-3) / 1e9 / pk["hbm_gbs"]},
-                "clocks": res["clocks"],
-                "e2e": None if args.no_e2e else {
-                    "value": flops * args.steps / (res["e2e_ms"] * 1e-3) / 1e12, "unit": UNIT,
-                    "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
-                "gpu_launches": res["launches"],
-            }
-            if not args.no_cpu_baseline:
-                line["cpu_baseline"] = cpu_baseline()
             print(json.dumps(line), flush=True)
     finally:
         if world > 1:
