@@ -175,8 +175,10 @@ arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, con
     if ((st = launch_status()) != ARC_OK) return st;
     first = true;
   } else if (!static_scale) {
+    // a persistent streaming grid: four 256-thread CTAs per SM, each thread many 16-byte loads
     const int64_t items = M * ((K + arc::kAmaxSeg - 1) / arc::kAmaxSeg);
-    npartials = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((items + 7) / 8, arc::kMaxPartials)));
+    npartials = static_cast<int>(std::max<int64_t>(
+        1, std::min<int64_t>({(items + 7) / 8, static_cast<int64_t>(sms) * 4, arc::kMaxPartials})));
     arc::k_amax<<<static_cast<unsigned>(npartials), 256, 0, s>>>(xb, ldx, static_cast<int>(M), static_cast<int>(K),
                                                                 w.partials);
     if ((st = launch_status()) != ARC_OK) return st;

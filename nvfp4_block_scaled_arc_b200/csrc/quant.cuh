@@ -307,25 +307,41 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 
 constexpr int kAmaxSeg = 2048;  // elements of a row per warp work item
 
-// max |x| over X [M, K]: warps over (row, 2048-element segment) items, eight 16-byte loads in
-// flight per lane; one partial per CTA (fp32 bits of the magnitude).
+// max |x| over X [M, K], one partial per CTA (fp32 bits of the magnitude). Contiguous rows
+// (ldx == K) are streamed as one flat array, every thread eight 16-byte loads in flight per
+// round; otherwise warps take (row, 2048-element segment) items.
 __global__ void __launch_bounds__(256) k_amax(const __nv_bfloat16* __restrict__ x, int64_t ldx, int M, int K,
                                               uint32_t* partials) {
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nseg = (K + kAmaxSeg - 1) / kAmaxSeg;
-  const int64_t items = static_cast<int64_t>(M) * nseg;
   uint32_t mx = 0;
-  for (int64_t it = static_cast<int64_t>(blockIdx.x) * 8 + warp; it < items; it += static_cast<int64_t>(gridDim.x) * 8) {
-    const int m = static_cast<int>(it / nseg), seg = static_cast<int>(it - static_cast<int64_t>(m) * nseg);
-    const __nv_bfloat16* row = x + static_cast<int64_t>(m) * ldx;
-    const int k0 = seg * kAmaxSeg + 8 * lane;
-    const int k1 = min(K, (seg + 1) * kAmaxSeg);
-    uint4 w[8];
+  if (ldx == K) {
+    const int64_t chunks = static_cast<int64_t>(M) * (K >> 3);  // 8 elements each
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t c0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c0 < chunks; c0 += 8 * stride) {
+      uint4 w[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = (k0 + 256 * i < k1) ? ld_nc_v4(row + k0 + 256 * i) : make_uint4(0, 0, 0, 0);
+      for (int i = 0; i < 8; ++i) {
+        const int64_t c = c0 + i * stride;
+        w[i] = c < chunks ? ld_nc_v4(x + 8 * c) : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) mx = absmax_bf16x2(mx, w[i]);
+      for (int i = 0; i < 8; ++i) mx = absmax_bf16x2(mx, w[i]);
+    }
+  } else {
+    const int nseg = (K + kAmaxSeg - 1) / kAmaxSeg;
+    const int64_t items = static_cast<int64_t>(M) * nseg;
+    for (int64_t it = static_cast<int64_t>(blockIdx.x) * 8 + warp; it < items; it += static_cast<int64_t>(gridDim.x) * 8) {
+      const int m = static_cast<int>(it / nseg), seg = static_cast<int>(it - static_cast<int64_t>(m) * nseg);
+      const __nv_bfloat16* row = x + static_cast<int64_t>(m) * ldx;
+      const int k0 = seg * kAmaxSeg + 8 * lane;
+      const int k1 = min(K, (seg + 1) * kAmaxSeg);
+      uint4 w[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] = (k0 + 256 * i < k1) ? ld_nc_v4(row + k0 + 256 * i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx = absmax_bf16x2(mx, w[i]);
+    }
   }
   cta_max_to(max(mx & 0xFFFFu, mx >> 16) << 16, &partials[blockIdx.x]);
 }
@@ -358,6 +374,22 @@ __global__ void __launch_bounds__(kQRowThreads, 6) k_quant_rows(QuantArgs a, int
   float* stash = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(slots) +
                                           static_cast<size_t>(qrows_nslot(a.K, a.r)) * 48);
   __shared__ int nslot_sh;
+  // the first batch of a row's blocks is loaded while the previous row finishes its residual
+  // step, so each row starts with its data in flight; the first row's at entry, under the set-up
+  uint4 raw[kQRowDepth][2];
+  auto load_batch = [&](const __nv_bfloat16* rp, int b0) {
+#pragma unroll
+    for (int i = 0; i < kQRowDepth; ++i) {
+      const int b = b0 + NT * i + tid;
+      if (b < nblk) {
+        raw[i][0] = ld_nc_v4(rp + 16 * b);
+        raw[i][1] = ld_nc_v4(rp + 16 * b + 8);
+      } else {
+        raw[i][0] = raw[i][1] = make_uint4(0, 0, 0, 0);
+      }
+    }
+  };
+  if (static_cast<int>(blockIdx.x) < a.M) load_batch(a.x + static_cast<int64_t>(blockIdx.x) * a.ldx, 0);
 
   // outlier tables (before the wait: they overlap the first kernel); out-of-range entries are
   // reported and left out
@@ -410,17 +442,7 @@ __global__ void __launch_bounds__(kQRowThreads, 6) k_quant_rows(QuantArgs a, int
     if (RMS) inv = a.inv_rms[m];
     // ---- primary blocks: thread t codes blocks b0 + 128 i + t
     for (int b0 = 0; b0 < nblk; b0 += NT * kQRowDepth) {
-      uint4 raw[kQRowDepth][2];
-#pragma unroll
-      for (int i = 0; i < kQRowDepth; ++i) {
-        const int b = b0 + NT * i + tid;
-        if (b < nblk) {
-          raw[i][0] = ld_nc_v4(row + 16 * b);
-          raw[i][1] = ld_nc_v4(row + 16 * b + 8);
-        } else {
-          raw[i][0] = raw[i][1] = make_uint4(0, 0, 0, 0);
-        }
-      }
+      if (b0 > 0) load_batch(row, b0);
 #pragma unroll
       for (int i = 0; i < kQRowDepth; ++i) {
         const int b = b0 + NT * i + tid;
@@ -503,6 +525,10 @@ __global__ void __launch_bounds__(kQRowThreads, 6) k_quant_rows(QuantArgs a, int
           }
         }
       }
+    }
+    {
+      const int mn = m + static_cast<int>(gridDim.x);
+      if (mn < a.M) load_batch(a.x + static_cast<int64_t>(mn) * a.ldx, 0);
     }
     if (a.r > 0) {
       // ---- outlier channels: residual x - E2M1(code) * d (activations) or the value itself
