@@ -90,6 +90,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
+// Wait used only while tearing down after an abort: bounded by time, ignores the abort flag.
+__device__ __forceinline__ void mbar_wait_teardown(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_test(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) return;
+  }
+}
+
 // ---------------------------------------------------------------------------------------------
 // TMA (tiled tensor loads, no multicast) and 1-D bulk copies
 // ---------------------------------------------------------------------------------------------

@@ -118,13 +118,6 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
   tn = rr / gm;
 }
 
-// Wait used only while tearing down after an abort: bounded by time, ignores the abort flag.
-__device__ __forceinline__ void mbar_wait_teardown(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_test(bar, parity)) {
-    if (globaltimer_ns() - t0 > limit_ns) return;
-  }
-}
 
 __device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
   uint32_t v;
