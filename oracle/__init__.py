@@ -219,6 +219,15 @@ def calibrate(x, r: int) -> np.ndarray:
     return idx[:r].copy()
 
 
+def calibrate_order(x) -> np.ndarray:
+    """All K channels ordered by calibration abs-max, descending, ties by ascending index: the
+    channel reorder of ARCQuant's adaptive outlier identification ("reorders the channels by
+    their absolute maxima and selects a top-S subset", Methodologie). The first r entries are
+    calibrate(x, r)."""
+    x = as_u16(x)
+    return calibrate(x, x.shape[1])
+
+
 # --------------------------------------------------------------------------------------------
 # Quantization (arc_oracle.c: activation quantization with augmented residual channels)
 # --------------------------------------------------------------------------------------------
@@ -269,6 +278,32 @@ def pack_weight(w, idx, s_w: float):
 
     _split_rows(N, run, min_rows=16)
     return codes, sf
+
+
+def quantize_act_reordered(x, perm, r: int, s_t: float, rms_gain=None, use_rms: bool = False,
+                           eps: float = 1e-6, want_residual: bool = False):
+    """Dual-stage quantization of the reordered activation (ARCQuant, Methodologie: the primary
+    stage quantizes the reordered input block-wise, the residual stage the top-S outlier
+    channels). Primary channel p of the output is input channel perm[p]; the outlier channels
+    are perm[:r], i.e. the first r columns of the reordered X, so this is quantize_act of
+    X[:, perm] with idx = 0..r-1 (an RMSNorm gain is reordered with X; the row statistics do not
+    depend on the channel order)."""
+    x = as_u16(x)
+    perm = np.ascontiguousarray(np.asarray(perm, dtype=np.int64).reshape(-1))
+    assert perm.size == x.shape[1] and 0 <= r <= perm.size
+    g = None if rms_gain is None else as_u16(rms_gain).reshape(-1)[perm]
+    return quantize_act(np.ascontiguousarray(x[:, perm]), np.arange(r, dtype=np.int32), s_t, rms_gain=g,
+                        use_rms=use_rms, eps=eps, want_residual=want_residual)
+
+
+def pack_weight_reordered(w, perm, r: int, s_w: float):
+    """W_aug = [W[:, perm] | W[:, perm[:r]]] packed as NVFP4: the weight side of the reordered
+    augmented GEMM (ARCQuant, Methodologie: weights reordered like the activation and their
+    outlier columns duplicated)."""
+    w = as_u16(w)
+    perm = np.ascontiguousarray(np.asarray(perm, dtype=np.int64).reshape(-1))
+    assert perm.size == w.shape[1] and 0 <= r <= perm.size
+    return pack_weight(np.ascontiguousarray(w[:, perm]), np.arange(r, dtype=np.int32), s_w)
 
 
 def dequant(codes, sf) -> np.ndarray:
