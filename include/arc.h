@@ -116,8 +116,9 @@ size_t arc_calibrate_workspace_bytes(int64_t K);
  *   workspace       device scratch of arc_quantize_workspace_bytes(M, r) bytes, 256-byte aligned;
  *                   contents need not be initialised; calls sharing a workspace must be ordered.
  * Requires K % 16 == 0, r % 16 == 0, 0 <= r <= K, ldx >= K, x rows 16-byte aligned. The
- * residuals are staged in shared memory (about 210 bytes per outlier channel), which accepts
- * r <= 896 for any K <= 65536; larger requests return ARC_ERR_UNSUPPORTED.
+ * residuals are staged in shared memory (56 bytes per outlier channel plus K/8 bytes of block
+ * table, at most 200 KB), which accepts r <= 3504 for any K <= 65536 and r <= 1312 up to
+ * K = 2^20; larger requests return ARC_ERR_UNSUPPORTED.
  */
 arc_status arc_quantize_act_nvfp4(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, const int32_t* d_idx,
                                   int32_t r, const void* rms_gain_bf16, float rms_eps, const float* d_static_scale,
@@ -141,6 +142,46 @@ arc_status arc_pack_weight_nvfp4(const void* w_bf16, int64_t N, int64_t K, int64
  */
 arc_status arc_calibrate_outliers(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, int32_t r,
                                   int32_t* d_idx_out, void* workspace, size_t ws_bytes, arc_stream_t stream);
+
+/*
+ * Channel reorder ("Adaptieve Uitschieter-identificatie": the channels are reordered by their
+ * absolute maxima and a top-S subset is selected): all K channels of the calibration tensor
+ * X [M, K] in descending abs-max order, ties by ascending index, written to d_perm_out (device
+ * int32[K]); its first r entries are what arc_calibrate_outliers returns for r. Workspace as
+ * arc_calibrate_outliers. The ranking does O(K^2) comparisons on the device (a calibration
+ * step: about 0.1 ms at K = 28672). 0 < K <= 2^20, K even, x 4-byte aligned.
+ */
+arc_status arc_calibrate_order(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, int32_t* d_perm_out,
+                               void* workspace, size_t ws_bytes, arc_stream_t stream);
+
+/*
+ * Reordered dual-stage quantization ("Primaire Fase: de input-activatiematrix wordt geherordend
+ * en gekwantiseerd"; Kernel Implementatie: reordering, RMSNorm, primary and residual
+ * quantization in one kernel). Primary channel p of the output is input channel d_perm[p]; the
+ * r outlier channels are d_perm[0 .. r), so appended block j (columns K + 16 j ..) holds the
+ * residuals x - E2M1(code) * d of primary block j's channels, coded with the same tensor scale.
+ * The result equals arc_quantize_act_nvfp4 applied to X[:, perm] with idx = 0 .. r-1.
+ *   d_perm          device int32[K], a permutation of 0 .. K-1, 16-byte aligned (entries outside
+ *                   [0, K) are read as channel K-1; a repeated entry repeats that channel).
+ * Other arguments, layouts and workspace as arc_quantize_act_nvfp4 (the RMSNorm gain is indexed
+ * by input channel). Each row is staged in shared memory twice over: K <= 51200, else
+ * ARC_ERR_UNSUPPORTED.
+ */
+arc_status arc_quantize_act_nvfp4_reordered(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                                            const int32_t* d_perm, int32_t r, const void* rms_gain_bf16,
+                                            float rms_eps, const float* d_static_scale, uint8_t* codes, uint8_t* sf,
+                                            float* d_scale_out, void* workspace, size_t ws_bytes,
+                                            arc_stream_t stream);
+
+/*
+ * Weights of the reordered augmented GEMM: W_aug = [W[:, perm] | W[:, perm[0 .. r)]] packed as
+ * NVFP4 with one tensor scale s_W = amax(|W|)/2688; the appended blocks repeat primary blocks
+ * 0 .. r/16 - 1. Same requirements as arc_quantize_act_nvfp4_reordered (rows = N).
+ */
+arc_status arc_pack_weight_nvfp4_reordered(const void* w_bf16, int64_t N, int64_t K, int64_t ldw,
+                                           const int32_t* d_perm, int32_t r, uint8_t* codes, uint8_t* sf,
+                                           float* d_scale_out, void* workspace, size_t ws_bytes,
+                                           arc_stream_t stream);
 
 /* ----------------------------------------------------------------------------------------- */
 /* GEMMs ("Unified GEMM Executie"; RAMP's BF16 reference path)                                 */

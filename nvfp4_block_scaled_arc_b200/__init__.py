@@ -61,6 +61,17 @@ _SIGS = {
     "arc_calibrate_outliers": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                               ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                               ctypes.c_void_p]),
+    "arc_calibrate_order": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "arc_quantize_act_nvfp4_reordered": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                                        ctypes.c_int64, ctypes.c_void_p, ctypes.c_int32,
+                                                        ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p,
+                                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                        ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "arc_pack_weight_nvfp4_reordered": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                                       ctypes.c_int64, ctypes.c_void_p, ctypes.c_int32,
+                                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                       ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "arc_gemm_nvfp4": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                       ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64,
@@ -210,6 +221,56 @@ def calibrate_outliers(x: torch.Tensor, r: int, stream=None) -> torch.Tensor:
     _check("arc_calibrate_outliers", lib().arc_calibrate_outliers(_p(x), M, K, x.stride(0), r, _p(idx), _p(ws),
                                                                   ws.numel(), _stream(stream)))
     return idx
+
+
+def calibrate_order(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """arc_calibrate_order: all K channels of X by descending abs-max (device int32[K])."""
+    _need_cuda(x)
+    M, K = x.shape
+    perm = torch.empty(K, dtype=torch.int32, device=x.device)
+    ws = _ws(int(lib().arc_calibrate_workspace_bytes(K)), x.device)
+    _check("arc_calibrate_order", lib().arc_calibrate_order(_p(x), M, K, x.stride(0), _p(perm), _p(ws), ws.numel(),
+                                                            _stream(stream)))
+    return perm
+
+
+def quantize_act_nvfp4_reordered(x: torch.Tensor, perm: torch.Tensor, r: int, rms_gain: torch.Tensor | None = None,
+                                 eps: float = 1e-6, static_scale: torch.Tensor | None = None,
+                                 out: NVFP4Tensor | None = None, workspace: torch.Tensor | None = None,
+                                 stream=None) -> NVFP4Tensor:
+    """arc_quantize_act_nvfp4_reordered: X [M, K] bf16 -> NVFP4 of X[:, perm] with the residuals of
+    the r channels perm[:r] appended."""
+    _need_cuda(x, perm, rms_gain, static_scale)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    assert perm.dtype == torch.int32 and perm.numel() == x.shape[1]
+    M, K = x.shape
+    if out is None:
+        out = NVFP4Tensor(_u8(codes_bytes(M, K + r), x.device), _u8(sf_bytes(M, K + r), x.device),
+                          torch.empty(1, dtype=torch.float32, device=x.device), M, K + r)
+    if workspace is None:
+        workspace = _ws(quantize_workspace_bytes(M, r), x.device)
+    _check("arc_quantize_act_nvfp4_reordered", lib().arc_quantize_act_nvfp4_reordered(
+        _p(x), M, K, x.stride(0), _p(perm), int(r), _p(rms_gain), float(eps), _p(static_scale), _p(out.codes),
+        _p(out.sf), _p(out.scale), _p(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
+def pack_weight_nvfp4_reordered(w: torch.Tensor, perm: torch.Tensor, r: int, out: NVFP4Tensor | None = None,
+                                workspace: torch.Tensor | None = None, stream=None) -> NVFP4Tensor:
+    """arc_pack_weight_nvfp4_reordered: W [N, K] bf16 -> NVFP4 of [W[:, perm] | W[:, perm[:r]]]."""
+    _need_cuda(w, perm)
+    assert w.dtype == torch.bfloat16 and w.dim() == 2 and w.stride(1) == 1
+    assert perm.dtype == torch.int32 and perm.numel() == w.shape[1]
+    N, K = w.shape
+    if out is None:
+        out = NVFP4Tensor(_u8(codes_bytes(N, K + r), w.device), _u8(sf_bytes(N, K + r), w.device),
+                          torch.empty(1, dtype=torch.float32, device=w.device), N, K + r)
+    if workspace is None:
+        workspace = _ws(quantize_workspace_bytes(N, r), w.device)
+    _check("arc_pack_weight_nvfp4_reordered", lib().arc_pack_weight_nvfp4_reordered(
+        _p(w), N, K, w.stride(0), _p(perm), int(r), _p(out.codes), _p(out.sf), _p(out.scale), _p(workspace),
+        workspace.numel(), _stream(stream)))
+    return out
 
 
 def gemm_nvfp4(a: NVFP4Tensor, b: NVFP4Tensor, out: torch.Tensor | None = None, add: torch.Tensor | None = None,

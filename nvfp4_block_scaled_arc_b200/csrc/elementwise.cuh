@@ -75,6 +75,29 @@ __global__ void __launch_bounds__(256) k_colmax(const __nv_bfloat16* __restrict_
   if (mx >> 16) atomicMax(&colmax[2 * kp + 1], mx & 0xFFFF0000u);
 }
 
+// Full calibration order (the channel reorder of ARCQuant's adaptive outlier identification):
+// channel c goes to position rank(c) = #{c' : key(c') > key(c)}, key = (abs-max bits << 32) |
+// (2^32 - 1 - c), i.e. larger abs-max first and ties by ascending channel. The keys are distinct,
+// so the ranks form a permutation and no two threads write the same slot. O(K^2) comparisons
+// through shared-memory tiles that every thread of the CTA reads in the same order (broadcast);
+// a calibration step, not part of the per-batch path.
+__global__ void __launch_bounds__(256) k_order(const uint32_t* colmax, int K, int32_t* perm_out) {
+  __shared__ uint64_t tile[2048];
+  const int c = blockIdx.x * 256 + threadIdx.x;
+  const uint64_t mine = c < K ? (static_cast<uint64_t>(colmax[c]) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(c)) : 0;
+  int rank = 0;
+  for (int t0 = 0; t0 < K; t0 += 2048) {
+    const int n = min(2048, K - t0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += 256)
+      tile[i] = (static_cast<uint64_t>(colmax[t0 + i]) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(t0 + i));
+    __syncthreads();
+#pragma unroll 8
+    for (int i = 0; i < n; ++i) rank += tile[i] > mine ? 1 : 0;
+  }
+  if (c < K) perm_out[rank] = c;
+}
+
 // Top-r channels by abs-max (descending), ties by ascending index, r rounds of a block-wide
 // argmax over 64-bit keys (abs-max bits << 32 | ~index).
 __global__ void __launch_bounds__(1024) k_topk(const uint32_t* colmax, int K, int r, uint64_t* keys, int32_t* idx_out) {

@@ -59,7 +59,11 @@ arc_status device_check(int* sms) {
         cudaFuncSetAttribute(arc::k_quant_rows<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              arc::kQRowsSmemMax) != cudaSuccess ||
         cudaFuncSetAttribute(arc::k_quant_rows<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             arc::kQRowsSmemMax) != cudaSuccess)
+                             arc::kQRowsSmemMax) != cudaSuccess ||
+        cudaFuncSetAttribute(arc::k_quant_reordered<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             arc::kQReoSmemMax) != cudaSuccess ||
+        cudaFuncSetAttribute(arc::k_quant_reordered<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             arc::kQReoSmemMax) != cudaSuccess)
       return ARC_ERR_CUDA;
     d.attrs_set = true;
   }
@@ -145,16 +149,21 @@ QuantWs carve_quant_ws(void* ws) {
   return w;
 }
 
+// Quantization driver shared by activations and weights, in the natural channel order (idx lists
+// the outlier channels) or reordered (perm != nullptr: primary channel p is input channel perm[p]
+// and the outlier channels are perm[0 .. r)).
 arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, const int32_t* idx, int32_t r,
                            const void* gain, float eps, const float* static_scale, uint8_t* codes, uint8_t* sf,
-                           float* scale_out, void* workspace, size_t ws_bytes, arc_stream_t stream, int dup) {
+                           float* scale_out, void* workspace, size_t ws_bytes, arc_stream_t stream, int dup,
+                           const int32_t* perm = nullptr) {
   if (!x || !codes || !sf || !scale_out) return ARC_ERR_INVALID_ARG;
   if (M <= 0 || K <= 0 || K % 16 || r < 0 || r % 16 || r > K || ldx < K) return ARC_ERR_INVALID_ARG;
-  if (r > 0 && !idx) return ARC_ERR_INVALID_ARG;
+  if (!perm && r > 0 && !idx) return ARC_ERR_INVALID_ARG;
   if (M > (1ll << 30) || K > (1ll << 20) || r > 32767) return ARC_ERR_UNSUPPORTED;
-  const size_t smem = arc::qrows_smem_bytes(static_cast<int>(K), r);
-  if (smem > static_cast<size_t>(arc::kQRowsSmemMax)) return ARC_ERR_UNSUPPORTED;
-  if (!al16(x) || (ldx * 2) % 16 || !al16(codes) || !al16(sf) || (gain && !al16(gain))) return ARC_ERR_ALIGNMENT;
+  const size_t smem = perm ? arc::qreo_smem_bytes(static_cast<int>(K)) : arc::qrows_smem_bytes(static_cast<int>(K), r);
+  if (smem > static_cast<size_t>(perm ? arc::kQReoSmemMax : arc::kQRowsSmemMax)) return ARC_ERR_UNSUPPORTED;
+  if (!al16(x) || (ldx * 2) % 16 || !al16(codes) || !al16(sf) || (gain && !al16(gain)) || (perm && !al16(perm)))
+    return ARC_ERR_ALIGNMENT;
   if (!workspace || ws_bytes < arc_quantize_workspace_bytes(M, r)) return ARC_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ARC_ERR_ALIGNMENT;
   int sms = 0;
@@ -202,7 +211,30 @@ arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, con
   a.codes = codes;
   a.sf = sf;
   a.dup = dup;
+  a.wait_ns = g_wait_ns;
   const int mpad = static_cast<int>((M + 127) / 128 * 128);
+  // the second launch may begin while the first one runs; it waits for the first one's results
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  if (perm) {
+    const void* rk = gain ? reinterpret_cast<const void*>(arc::k_quant_reordered<true>)
+                          : reinterpret_cast<const void*>(arc::k_quant_reordered<false>);
+    int rper_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&rper_sm, rk, arc::kQReoThreads, smem) != cudaSuccess ||
+        rper_sm < 1)
+      return ARC_ERR_CUDA;
+    cudaLaunchConfig_t rc = {};
+    rc.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(mpad, static_cast<int64_t>(sms) * rper_sm)));
+    rc.blockDim = dim3(arc::kQReoThreads);
+    rc.dynamicSmemBytes = smem;
+    rc.stream = s;
+    rc.attrs = pdl;
+    rc.numAttrs = first ? 1 : 0;
+    const cudaError_t re = gain ? cudaLaunchKernelEx(&rc, arc::k_quant_reordered<true>, a, perm, mpad)
+                                : cudaLaunchKernelEx(&rc, arc::k_quant_reordered<false>, a, perm, mpad);
+    return re == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
+  }
   const void* kern = gain ? reinterpret_cast<const void*>(arc::k_quant_rows<true>)
                           : reinterpret_cast<const void*>(arc::k_quant_rows<false>);
   int per_sm = 0;
@@ -328,6 +360,48 @@ arc_status arc_calibrate_outliers(const void* x_bf16, int64_t M, int64_t K, int6
   if ((st = launch_status()) != ARC_OK) return st;
   arc::k_topk<<<1, 1024, 0, s>>>(colmax, static_cast<int>(K), r, keys, d_idx_out);
   return launch_status();
+}
+
+arc_status arc_calibrate_order(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, int32_t* d_perm_out,
+                               void* workspace, size_t ws_bytes, arc_stream_t stream) {
+  if (!x_bf16 || !d_perm_out) return ARC_ERR_INVALID_ARG;
+  if (M <= 0 || K <= 0 || K % 2 || ldx < K) return ARC_ERR_INVALID_ARG;
+  if (M > (1ll << 30) || K > (1ll << 20)) return ARC_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(x_bf16) & 3u) || ldx % 2) return ARC_ERR_ALIGNMENT;
+  if (!workspace || ws_bytes < arc_calibrate_workspace_bytes(K)) return ARC_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ARC_ERR_ALIGNMENT;
+  int sms = 0;
+  arc_status st = device_check(&sms);
+  if (st != ARC_OK) return st;
+  cudaStream_t s = S(stream);
+  uint32_t* colmax = static_cast<uint32_t*>(workspace);
+  if (cudaMemsetAsync(colmax, 0, static_cast<size_t>(K) * 4, s) != cudaSuccess) return ARC_ERR_CUDA;
+  const int rows_per_cta = 64;
+  dim3 grid(static_cast<unsigned>((K / 2 + 255) / 256), static_cast<unsigned>((M + rows_per_cta - 1) / rows_per_cta));
+  arc::k_colmax<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x_bf16), ldx, static_cast<int>(M),
+                                     static_cast<int>(K), rows_per_cta, colmax);
+  if ((st = launch_status()) != ARC_OK) return st;
+  arc::k_order<<<static_cast<unsigned>((K + 255) / 256), 256, 0, s>>>(colmax, static_cast<int>(K), d_perm_out);
+  return launch_status();
+}
+
+arc_status arc_quantize_act_nvfp4_reordered(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                                            const int32_t* d_perm, int32_t r, const void* rms_gain_bf16,
+                                            float rms_eps, const float* d_static_scale, uint8_t* codes, uint8_t* sf,
+                                            float* d_scale_out, void* workspace, size_t ws_bytes,
+                                            arc_stream_t stream) {
+  if (!d_perm) return ARC_ERR_INVALID_ARG;
+  return quantize_common(x_bf16, M, K, ldx, nullptr, r, rms_gain_bf16, rms_eps, d_static_scale, codes, sf,
+                         d_scale_out, workspace, ws_bytes, stream, 0, d_perm);
+}
+
+arc_status arc_pack_weight_nvfp4_reordered(const void* w_bf16, int64_t N, int64_t K, int64_t ldw,
+                                           const int32_t* d_perm, int32_t r, uint8_t* codes, uint8_t* sf,
+                                           float* d_scale_out, void* workspace, size_t ws_bytes,
+                                           arc_stream_t stream) {
+  if (!d_perm) return ARC_ERR_INVALID_ARG;
+  return quantize_common(w_bf16, N, K, ldw, nullptr, r, nullptr, 0.0f, nullptr, codes, sf, d_scale_out, workspace,
+                         ws_bytes, stream, 1, d_perm);
 }
 
 arc_status arc_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_sf, const float* d_a_scale,

@@ -47,6 +47,7 @@ struct QuantArgs {
   uint8_t* codes;
   uint8_t* sf;
   int dup;       // 1: weights (stash the value itself), 0: activations (stash the residual)
+  uint64_t wait_ns;  // bound on the reordered kernel's waits (one that runs out sets the timeout status)
 };
 
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
@@ -579,6 +580,229 @@ __global__ void __launch_bounds__(kQRowThreads, 6) k_quant_rows(QuantArgs a, int
       const int kb = nblk + rb;
       sf_row[(kb >> 2) * 512 + (kb & 3)] = static_cast<uint8_t>(sfv);
     }
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Reordered quantization (ARCQuant, Methodologie: "the input activation matrix is reordered and
+// quantized with standard block-wise NVFP4"; Kernel Implementatie: one fused kernel for channel
+// reordering, RMSNorm, primary and residual quantization). Primary block b holds input channels
+// perm[16 b .. 16 b + 15]; the outlier channels are perm[0 .. r), i.e. exactly the channels of
+// primary blocks 0 .. r/16 - 1, so appended block j is formed from primary block j: its residuals
+// x - E2M1(code) * d (activations) or, for weights, the same 16 values, which code to the same
+// bytes as the primary block.
+// ---------------------------------------------------------------------------------------------
+
+constexpr int kQReoThreads = 256;
+constexpr int kQReoSmemMax = 200 * 1024;  // two row buffers: K <= 51200 channels
+
+__host__ __device__ constexpr size_t qreo_row_bytes(int K) { return (static_cast<size_t>(K) * 2 + 127) / 128 * 128; }
+__host__ __device__ constexpr size_t qreo_smem_bytes(int K) { return 2 * qreo_row_bytes(K); }
+
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t ldg_nc_u16(const void* p) {
+  uint16_t v;
+  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+
+// One CTA codes one row at a time; rows arrive by 1-D bulk copies into two shared-memory
+// buffers (the next row loads while this one is coded). Thread t codes primary blocks t, t + 256,
+// ..., gathering its 16 channels from the row buffer through perm; threads whose block is below
+// r/16 then code the appended block of the same channels from the values, codes and d they hold.
+template <bool RMS>
+__global__ void __launch_bounds__(kQReoThreads, 3) k_quant_reordered(QuantArgs a, const int32_t* __restrict__ perm,
+                                                                     int mpad) {
+  extern __shared__ __align__(128) uint8_t qreo_smem[];
+  constexpr int NT = kQReoThreads;
+  const int nblk = a.K >> 4;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const size_t rowb = qreo_row_bytes(a.K);
+  __shared__ uint64_t row_full[2];
+  __shared__ volatile int abort_sh;
+  const int nrows_mine = static_cast<int>(blockIdx.x) < a.M
+                             ? (a.M - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                             : 0;
+  uint32_t armed = 0;  // thread 0: row buffers with a copy issued and not yet waited for
+  auto issue = [&](int it) {
+    const int64_t m = static_cast<int64_t>(blockIdx.x) + static_cast<int64_t>(it) * gridDim.x;
+    const int buf = it & 1;
+    const uint32_t bytes = static_cast<uint32_t>(a.K) * 2u;
+    mbar_arrive_expect_tx(&row_full[buf], bytes);
+    bulk_load(qreo_smem + buf * rowb, a.x + m * a.ldx, bytes, &row_full[buf]);
+    armed |= 1u << buf;
+  };
+  // X is only read by the earlier kernel, so the first rows may load before the programmatic wait
+  if (tid == 0) {
+    mbar_init(&row_full[0], 1);
+    mbar_init(&row_full[1], 1);
+    abort_sh = 0;
+    fence_mbar_init();
+    if (nrows_mine > 0) issue(0);
+    if (nrows_mine > 1) issue(1);
+  }
+  __syncthreads();
+
+  // ---- tensor scale and the decode scale table
+  pdl_wait();
+  float s;
+  {
+    __shared__ float s_sh;
+    s = a.static_scale ? *a.static_scale : cta_tensor_scale(a);
+    if (tid == 0) s_sh = s;
+    __syncthreads();
+    s = s_sh;
+  }
+  if (blockIdx.x == 0 && tid == 0) *a.scale_out = s;
+  const float rcp_s = __frcp_rn(s), rcp6 = __frcp_rn(6.0f);
+  __shared__ float2 dtab[128];
+  if (tid < 128) {
+    const float dd = __fmul_rn(e4m3_value(static_cast<uint32_t>(tid)), s);
+    dtab[tid] = make_float2(dd, in_safe_range(dd) ? -__frcp_rn(dd) : 0.0f);
+  }
+  __syncthreads();
+  const int64_t cpitch = a.kpad >> 1;
+  const int nres = a.r >> 4, ntail = (a.kpad - a.K) >> 4;
+
+  // rows padding the scale layout to a multiple of 128 carry zero scales
+  for (int m = a.M + static_cast<int>(blockIdx.x); m < mpad; m += gridDim.x)
+    for (int kb = tid; kb < (a.kpad >> 4); kb += NT) a.sf[sf_offset(m, kb, a.katoms)] = 0;
+
+  bool ok = true;
+  int it = 0;
+  for (; it < nrows_mine; ++it) {
+    const int64_t m = static_cast<int64_t>(blockIdx.x) + static_cast<int64_t>(it) * gridDim.x;
+    const int buf = it & 1;
+    const bool got = mbar_wait(&row_full[buf], static_cast<uint32_t>((it >> 1) & 1), a.wait_ns, &abort_sh);
+    if (!__syncthreads_and(got)) {
+      ok = false;
+      break;
+    }
+    const uint32_t srow = smem_u32(qreo_smem + buf * rowb);
+    const unsigned kmax = static_cast<unsigned>(a.K - 1);
+    uint8_t* crow = a.codes + m * cpitch;
+    double inv = 0.0;
+    if (RMS) inv = a.inv_rms[m];
+    for (int b0 = 0; b0 < nblk; b0 += NT) {
+      if (b0 + (tid & ~31) >= nblk) break;  // warp-uniform: the whole warp is past the end
+      const int b = b0 + tid;
+      const bool valid = b < nblk;
+      uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0}, gs[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      if (valid) {
+        const int4* pp = reinterpret_cast<const int4*>(perm + 16 * b);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          // a caller's out-of-range entry is clamped to the last channel (never read out of bounds)
+          int4 c = __ldg(pp + q);
+          c.x = static_cast<int>(min(static_cast<unsigned>(c.x), kmax));
+          c.y = static_cast<int>(min(static_cast<unsigned>(c.y), kmax));
+          c.z = static_cast<int>(min(static_cast<unsigned>(c.z), kmax));
+          c.w = static_cast<int>(min(static_cast<unsigned>(c.w), kmax));
+          w[2 * q] = lds_u16(srow + 2 * c.x) | (lds_u16(srow + 2 * c.y) << 16);
+          w[2 * q + 1] = lds_u16(srow + 2 * c.z) | (lds_u16(srow + 2 * c.w) << 16);
+          if (RMS) {
+            gs[2 * q] = ldg_nc_u16(a.gain + c.x) | (ldg_nc_u16(a.gain + c.y) << 16);
+            gs[2 * q + 1] = ldg_nc_u16(a.gain + c.z) | (ldg_nc_u16(a.gain + c.w) << 16);
+          }
+        }
+      }
+      float v[16];
+      float amax;
+      if constexpr (RMS) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          v[2 * e] = rms_apply(bf16_lo(w[e]), inv, bf16_lo(gs[e]));
+          v[2 * e + 1] = rms_apply(bf16_hi(w[e]), inv, bf16_hi(gs[e]));
+        }
+        const float a0 = fmax3_abs(v[0], v[1], v[2]), a1 = fmax3_abs(v[3], v[4], v[5]),
+                    a2 = fmax3_abs(v[6], v[7], v[8]), a3 = fmax3_abs(v[9], v[10], v[11]),
+                    a4 = fmax3_abs(v[12], v[13], v[14]);
+        amax = fmaxf(fmax3(a0, a1, a2), fmax3(a3, a4, fabsf(v[15])));
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          v[2 * e] = bf16_lo(w[e]);
+          v[2 * e + 1] = bf16_hi(w[e]);
+        }
+        const uint32_t m01 = __vmaxu2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu);
+        const uint32_t m23 = __vmaxu2(w[2] & 0x7FFF7FFFu, w[3] & 0x7FFF7FFFu);
+        const uint32_t m45 = __vmaxu2(w[4] & 0x7FFF7FFFu, w[5] & 0x7FFF7FFFu);
+        const uint32_t m67 = __vmaxu2(w[6] & 0x7FFF7FFFu, w[7] & 0x7FFF7FFFu);
+        const uint32_t mw = __vmaxu2(__vmaxu2(m01, m23), __vmaxu2(m45, m67));
+        amax = __uint_as_float(max(mw & 0xFFFFu, mw >> 16) << 16);
+      }
+      const uint32_t sfv = block_sf(amax, s, rcp_s, rcp6);
+      const float2 dn = dtab[sfv];
+      uint2 cc = make_uint2(0u, 0u);
+      if (dn.x != 0.0f) {
+        uint64_t p[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) p[e] = f2_pack(v[2 * e], v[2 * e + 1]);
+        cc = encode16_nr(p, dn.x, dn.y);
+      }
+      if (valid) *reinterpret_cast<uint2*>(crow + 8 * b) = cc;
+      // scale bytes: lanes 4i..4i+3 hold blocks b..b+3 (b % 4 == 0 at lane 4i)
+      const uint32_t my = valid ? sfv : 0u;
+      const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, my, 1), s2 = __shfl_down_sync(0xFFFFFFFFu, my, 2),
+                     s3 = __shfl_down_sync(0xFFFFFFFFu, my, 3);
+      if (valid && (lane & 3) == 0) {
+        uint8_t* dst = a.sf + sf_offset(m, b, a.katoms);
+        if (b + 3 < nblk) {
+          *reinterpret_cast<uint32_t*>(dst) = my | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        } else {
+          dst[0] = static_cast<uint8_t>(my);
+          if (b + 1 < nblk) dst[1] = static_cast<uint8_t>(s1);
+          if (b + 2 < nblk) dst[2] = static_cast<uint8_t>(s2);
+        }
+      }
+      // ---- the appended block of the same 16 channels
+      if (valid && b < nres) {
+        uint32_t rsf = sfv;
+        uint2 rc = cc;
+        if (!a.dup) {
+          float res[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const uint32_t code = (((e < 8) ? cc.x : cc.y) >> (4 * (e & 7))) & 15u;
+            res[e] = __fsub_rn(v[e], __fmul_rn(e2m1_value(code), dn.x));
+          }
+          const float a0 = fmax3_abs(res[0], res[1], res[2]), a1 = fmax3_abs(res[3], res[4], res[5]),
+                      a2 = fmax3_abs(res[6], res[7], res[8]), a3 = fmax3_abs(res[9], res[10], res[11]),
+                      a4 = fmax3_abs(res[12], res[13], res[14]);
+          rsf = block_sf(fmaxf(fmax3(a0, a1, a2), fmax3(a3, a4, fabsf(res[15]))), s, rcp_s, rcp6);
+          const float2 rn = dtab[rsf];
+          rc = make_uint2(0u, 0u);
+          if (rn.x != 0.0f) {
+            uint64_t p[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) p[e] = f2_pack(res[2 * e], res[2 * e + 1]);
+            rc = encode16_nr(p, rn.x, rn.y);
+          }
+        }
+        *reinterpret_cast<uint2*>(crow + ((a.K + 16 * b) >> 1)) = rc;
+        a.sf[sf_offset(m, nblk + b, a.katoms)] = static_cast<uint8_t>(rsf);
+      }
+    }
+    // zero blocks padding the row to K_pad
+    for (int tb = nres + tid; tb < ntail; tb += NT) {
+      *reinterpret_cast<uint2*>(crow + ((a.K + 16 * tb) >> 1)) = make_uint2(0u, 0u);
+      a.sf[sf_offset(m, nblk + tb, a.katoms)] = 0;
+    }
+    // every thread is done with this buffer: load the row two ahead into it
+    __syncthreads();
+    if (tid == 0) {
+      armed &= ~(1u << buf);
+      if (it + 2 < nrows_mine) issue(it + 2);
+    }
+  }
+  // a wait that gave up leaves copies in flight: let them land before the CTA goes away
+  if (tid == 0 && !ok) {
+    for (int j = it; j < it + 2 && j < nrows_mine; ++j)
+      if ((armed >> (j & 1)) & 1u) mbar_wait_teardown(&row_full[j & 1], static_cast<uint32_t>((j >> 1) & 1), a.wait_ns);
   }
 }
 
