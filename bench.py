@@ -216,7 +216,16 @@ def run_layers(args, rank, world, device, layers, with_error=False):
     import workloads as W
 
     stream = torch.cuda.Stream(device=device)
+    reorder = getattr(args, "reorder", False)
     xs_host, xs, idx, packed, qa, ys, wsp, errs = {}, {}, {}, {}, {}, {}, {}, {}
+    rs = {L["name"]: L["r"] for L in layers}
+
+    def quant(name, **kw):
+        # the step's quantizer: natural channel order with the outlier list, or the reordered one
+        if reorder:
+            return arc.quantize_act_nvfp4_reordered(xs[name], idx[name], rs[name], stream=stream, **kw)
+        return arc.quantize_act_nvfp4(xs[name], idx[name], stream=stream, **kw)
+
     with torch.cuda.stream(stream):
         for L in layers:
             name, M, r = L["name"], L["M"], L["r"]
@@ -224,9 +233,14 @@ def run_layers(args, rank, world, device, layers, with_error=False):
             xs_host[name] = W.to_torch_bf16(d["x"])
             xs[name] = xs_host[name].to(device)
             w = W.to_torch_bf16(d["w"]).to(device)
-            idx[name] = arc.calibrate_outliers(xs[name], r, stream=stream) if r else None
-            packed[name] = arc.pack_weight_nvfp4(w, idx[name], stream=stream)
-            qa[name] = arc.quantize_act_nvfp4(xs[name], idx[name], stream=stream)
+            if reorder:
+                # idx holds the full calibration order; its first r channels are the outliers
+                idx[name] = arc.calibrate_order(xs[name], stream=stream)
+                packed[name] = arc.pack_weight_nvfp4_reordered(w, idx[name], r, stream=stream)
+            else:
+                idx[name] = arc.calibrate_outliers(xs[name], r, stream=stream) if r else None
+                packed[name] = arc.pack_weight_nvfp4(w, idx[name], stream=stream)
+            qa[name] = quant(name)
             ys[name] = torch.empty(M, L["N"], dtype=torch.bfloat16, device=device)
             wsp[name] = torch.empty(arc.quantize_workspace_bytes(M, r), dtype=torch.uint8, device=device)
             if with_error:
@@ -244,7 +258,7 @@ def run_layers(args, rank, world, device, layers, with_error=False):
             e0, e1, e2 = (_ev(), _ev(), _ev()) if rec is not None else (None, None, None)
             if e0 is not None:
                 e0.record(stream)
-            arc.quantize_act_nvfp4(xs[name], idx[name], out=qa[name], workspace=wsp[name], stream=stream)
+            quant(name, out=qa[name], workspace=wsp[name])
             if e1 is not None:
                 e1.record(stream)
             arc.gemm_nvfp4(qa[name], packed[name], out=ys[name], stream=stream)
@@ -303,7 +317,7 @@ def run_layers(args, rank, world, device, layers, with_error=False):
             for L in layers:
                 name = L["name"]
                 xs[name].copy_(xs_pin[name], non_blocking=True)
-                arc.quantize_act_nvfp4(xs[name], idx[name], out=qa[name], workspace=wsp[name], stream=stream)
+                quant(name, out=qa[name], workspace=wsp[name])
                 arc.gemm_nvfp4(qa[name], packed[name], out=ys[name], stream=stream)
                 ys_pin[name].copy_(ys[name], non_blocking=True)
 
@@ -346,7 +360,9 @@ def layers_line(args, world, layers, desc, res):
         "scaling": "weak", "vs_baseline": None, "dtype": "e2m1 x e2m1 -> f32 (bf16 out)",
         "data": "synthetic (seeded; random weights and activations of the stated shapes)",
         "config": {"workload": desc, "l2": "flushed (256 MiB write) before every step",
-                   "parallelism": f"replicas x{world}"},
+                   "parallelism": f"replicas x{world}",
+                   "channel_order": "reordered by calibration abs-max" if getattr(args, "reorder", False)
+                   else "natural (outlier list)"},
         "quant_gbs": quant_gbs,
         "gemm_only_tflops": achieved,
         "pct_fp4_peak": 100.0 * value / peak,
@@ -355,8 +371,12 @@ def layers_line(args, world, layers, desc, res):
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{src} bf16 burst {pk['bf16_tflops']} TFLOP/s x {FP4_OVER_BF16:g} "
                                     f"(nominal FP4/BF16 dense ratio)",
-                     "traffic": ncu_traffic() if args.workload == "llama8b" else None},
-        "quant_roofline": {"bound": "hbm", "kernel": "k_amax + k_quant_rows", "achieved": quant_gbs,
+                     "traffic": ncu_traffic() if args.workload == "llama8b" and not getattr(args, "reorder", False)
+                     else None},
+        "quant_roofline": {"bound": "hbm",
+                           "kernel": "k_amax + " + ("k_quant_reordered" if getattr(args, "reorder", False)
+                                                    else "k_quant_rows"),
+                           "achieved": quant_gbs,
                            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": quant_gbs / pk["hbm_gbs"],
                            "peak_source": f"{src} copy bandwidth"},
         "clocks": res["clocks"],
@@ -472,18 +492,22 @@ def run_recurrent(args, rank, world, device):
 # Oracle arm (CPU)
 # ---------------------------------------------------------------------------------------------
 
-def oracle_cache(layers, n_rows: int):
+def oracle_cache(layers, n_rows: int, reorder: bool = False):
     import oracle as O
 
     cache = {}
     for L in layers:
         d = L["gen"](n_rows, 0)
         x = d["x"][:n_rows]
-        idx = O.calibrate(x, L["r"]) if L["r"] else np.zeros(0, np.int32)
         sa = O.tensor_scale(O.amax(x))
         sw = O.tensor_scale(O.amax(d["w"]))
-        bc, bsf = O.pack_weight(d["w"], idx, sw)  # every output column needs the full weight
-        cache[L["name"]] = dict(x=x, idx=idx, sa=sa, sw=sw, bc=bc, bsf=bsf)
+        if reorder:
+            idx = O.calibrate_order(x)
+            bc, bsf = O.pack_weight_reordered(d["w"], idx, L["r"], sw)
+        else:
+            idx = O.calibrate(x, L["r"]) if L["r"] else np.zeros(0, np.int32)
+            bc, bsf = O.pack_weight(d["w"], idx, sw)  # every output column needs the full weight
+        cache[L["name"]] = dict(x=x, idx=idx, sa=sa, sw=sw, bc=bc, bsf=bsf, reorder=reorder)
     return cache
 
 
@@ -496,19 +520,22 @@ def oracle_sample_step(layers, rows: int, cache: dict):
     flops = 0.0
     for L in layers:
         c = cache[L["name"]]
-        ac, asf = O.quantize_act(c["x"][:rows], c["idx"], c["sa"])
+        if c["reorder"]:
+            ac, asf = O.quantize_act_reordered(c["x"][:rows], c["idx"], L["r"], c["sa"])
+        else:
+            ac, asf = O.quantize_act(c["x"][:rows], c["idx"], c["sa"])
         O.gemm_nvfp4_f64(ac, asf, c["sa"], c["bc"], c["bsf"], c["sw"])
         flops += 2.0 * rows * L["N"] * (L["K"] + L["r"])
     return flops
 
 
-def cpu_baseline(layers, rows: int | None = None):
+def cpu_baseline(layers, rows: int | None = None, reorder: bool = False):
     """The oracle on the host cores: `rows` token rows (default two per host thread, so every
     thread works) of each layer, about 10-30 s of CPU work."""
     import oracle as O
 
     rows = rows or 2 * O._threads()
-    cache = oracle_cache(layers, max(rows, 64))
+    cache = oracle_cache(layers, max(rows, 64), reorder)
     t0 = time.perf_counter()
     flops = oracle_sample_step(layers, rows, cache)
     dt = time.perf_counter() - t0
@@ -523,7 +550,7 @@ def run_reference(args, rank, world, layers, desc):
     import oracle as O
 
     rows = O._threads()  # one token row per host thread per step
-    cache = oracle_cache(layers, max(rows, 64))
+    cache = oracle_cache(layers, max(rows, 64), getattr(args, "reorder", False))
     for _ in range(args.warmup):
         oracle_sample_step(layers, rows, cache)
     t0 = time.perf_counter()
@@ -555,6 +582,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
     ap.add_argument("--proj", default="all", help="profiling: run only this layer (e.g. qkv, gateup)")
+    ap.add_argument("--reorder", action="store_true",
+                    help="linear-layer workloads: channels reordered by calibration abs-max before the primary "
+                         "quantization (the outlier set is the first r of the order)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -587,10 +617,11 @@ def main():
         if args.workload == "recurrent":
             line = run_recurrent(args, rank, world, device)
         else:
-            res = run_layers(args, rank, world, device, layers, with_error=args.workload == "stress")
+            res = run_layers(args, rank, world, device, layers,
+                             with_error=args.workload == "stress" or args.reorder)
             line = layers_line(args, world, layers, desc, res) if rank == 0 else None
             if rank == 0 and not args.no_cpu_baseline:
-                line["cpu_baseline"] = cpu_baseline(layers)
+                line["cpu_baseline"] = cpu_baseline(layers, reorder=args.reorder)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:
