@@ -472,6 +472,7 @@ def run_recurrent(args, rank, world, device):
                              "gemm_tflops": fl / (ms[k] * 1e-3) / 1e12,
                              "hidden_state_rel_err_vs_all_bf16": fidelity[k]}
     kk = 12 if 12 in ms else k_lows[-1]
+    study = schedule_study(arc, h, h0, blk, wsp, flush, stream, T, kk, out[0], device)
     # kernels per prefill: NVFP4 step = 2 x (2 quantizer launches + GEMM + SiLU + 2 quantizer
     # launches + GEMM), BF16 step = 2 x (RMSNorm + GEMM + SiLU + GEMM)
     launches = args.steps * sum(k * 2 * 7 + (T - k) * 2 * 4 for k in k_lows)
@@ -484,8 +485,45 @@ def run_recurrent(args, rank, world, device):
         "config": {"workload": f"recurrent SwiGLU block: S={S}, d={d}, ffn={F}, 2 pre-norm sublayers, T={T}, "
                                f"k_low in {k_lows}, r={r}",
                    "l2": "flushed (256 MiB write) before every prefill", "parallelism": f"replicas x{world}"},
-        "per_k_low": per, "clocks": clk.summary(), "e2e": None, "gpu_launches": launches,
+        "per_k_low": per, "schedule_study": study, "clocks": clk.summary(), "e2e": None, "gpu_launches": launches,
     }
+
+
+def schedule_study(arc, h, h0, blk, wsp, flush, stream, T, budget, ref, device, reps=5):
+    """Where the BF16 steps go at a fixed budget of NVFP4 steps (RAMP's matched-budget comparison:
+    low precision first and BF16 last, against Early-BF16 and random placements): hidden-state
+    error against all-BF16 and the prefill time of each schedule. Run after the timed region."""
+    rng = np.random.default_rng(3)
+    sch = {"ramp (NVFP4 first)": [1] * budget + [0] * (T - budget),
+           "early_bf16 (BF16 first)": [0] * (T - budget) + [1] * budget,
+           "interleaved": [0 if (t % (T // max(1, T - budget))) == T // max(1, T - budget) - 1 else 1
+                           for t in range(T)]}
+    for i in range(3):
+        f = np.zeros(T, np.int64)
+        f[rng.choice(T, size=budget, replace=False)] = 1
+        sch[f"random {i}"] = f.tolist()
+    res = {}
+    for name, flags in sch.items():
+        with torch.cuda.stream(stream):
+            h.copy_(h0)
+            arc.recurrent_prefill_schedule(h, blk, flags, workspace=wsp, stream=stream)
+            err = (torch.linalg.norm(h.float() - ref) / torch.linalg.norm(ref)).item()
+            ts = []
+            for _ in range(reps):
+                flush.zero_()
+                h.copy_(h0)
+                a, b = _ev(), _ev()
+                a.record(stream)
+                arc.recurrent_prefill_schedule(h, blk, flags, workspace=wsp, stream=stream)
+                b.record(stream)
+                ts.append((a, b))
+        stream.synchronize()
+        res[name] = {"schedule": "".join("L" if f else "B" for f in flags), "nvfp4_steps": int(sum(flags)),
+                     "ms": statistics.median(a.elapsed_time(b) for a, b in ts),
+                     "hidden_state_rel_err_vs_all_bf16": err}
+    if arc.last_device_status(stream) != 0:
+        raise RuntimeError("device status set during the schedule study")
+    return res
 
 
 # ---------------------------------------------------------------------------------------------

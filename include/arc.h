@@ -270,6 +270,17 @@ size_t arc_recurrent_workspace_bytes(int64_t S, const arc_swiglu_block* blk);
 arc_status arc_recurrent_prefill(void* h_bf16, int64_t S, const arc_swiglu_block* blk, int32_t T, int32_t k_low,
                                  void* workspace, size_t ws_bytes, arc_stream_t stream);
 
+/*
+ * The same recurrence with any per-step precision schedule (for schedule studies: RAMP's
+ * matched-budget comparison of where the BF16 steps go, "RAMP…" §6 and its Early-BF16 and
+ * random-schedule baselines): low_steps is a host array of T bytes, read during the call;
+ * step t runs in NVFP4 + ARC when low_steps[t] != 0, else in BF16. arc_recurrent_prefill with
+ * k_low is the schedule low_steps[t] = (t < k_low).
+ */
+arc_status arc_recurrent_prefill_schedule(void* h_bf16, int64_t S, const arc_swiglu_block* blk, int32_t T,
+                                          const uint8_t* low_steps, void* workspace, size_t ws_bytes,
+                                          arc_stream_t stream);
+
 /* ----------------------------------------------------------------------------------------- */
 /* Device status and failure detection                                                        */
 /* ----------------------------------------------------------------------------------------- */

@@ -88,6 +88,10 @@ _SIGS = {
     "arc_recurrent_prefill": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(SwigluBlock),
                                              ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t,
                                              ctypes.c_void_p]),
+    "arc_recurrent_prefill_schedule": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64,
+                                                      ctypes.POINTER(SwigluBlock), ctypes.c_int32,
+                                                      ctypes.POINTER(ctypes.c_uint8), ctypes.c_void_p,
+                                                      ctypes.c_size_t, ctypes.c_void_p]),
     "arc_last_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "arc_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64]),
     "arc_debug_inject": (ctypes.c_int, [ctypes.c_int32]),
@@ -349,6 +353,21 @@ def recurrent_prefill(h: torch.Tensor, block: RecurrentBlock, T: int, k_low: int
         workspace = _ws(n, h.device)
     _check("arc_recurrent_prefill", lib().arc_recurrent_prefill(_p(h), S, ctypes.byref(block.block), T, k_low,
                                                                 _p(workspace), workspace.numel(), _stream(stream)))
+    return h
+
+
+def recurrent_prefill_schedule(h: torch.Tensor, block: RecurrentBlock, schedule, workspace: torch.Tensor | None = None,
+                               stream=None) -> torch.Tensor:
+    """arc_recurrent_prefill_schedule: apply the block len(schedule) times in place; step t in
+    NVFP4 + ARC when schedule[t] is true, else in BF16."""
+    S = h.shape[0]
+    flags = (ctypes.c_uint8 * max(1, len(schedule)))(*[1 if f else 0 for f in schedule])
+    n = block.workspace_bytes(S)
+    if workspace is None:
+        workspace = _ws(n, h.device)
+    _check("arc_recurrent_prefill_schedule", lib().arc_recurrent_prefill_schedule(
+        _p(h), S, ctypes.byref(block.block), len(schedule), flags, _p(workspace), workspace.numel(),
+        _stream(stream)))
     return h
 
 

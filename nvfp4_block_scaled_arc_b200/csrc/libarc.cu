@@ -548,10 +548,12 @@ size_t arc_recurrent_workspace_bytes(int64_t S_, const arc_swiglu_block* blk) {
   return off[6] + arc_quantize_workspace_bytes(S_, rmax);
 }
 
-arc_status arc_recurrent_prefill(void* h_bf16, int64_t S_, const arc_swiglu_block* blk, int32_t T, int32_t k_low,
-                                 void* workspace, size_t ws_bytes, arc_stream_t stream) {
-  if (!h_bf16 || !blk || !blk->sublayers || blk->n_sublayers <= 0 || S_ <= 0 || T < 0 || k_low < 0)
-    return ARC_ERR_INVALID_ARG;
+// The recurrence with a per-step precision: step t runs in NVFP4 + ARC when low(t), else in BF16.
+extern "C++" {
+template <class Low>
+arc_status recurrent_run(void* h_bf16, int64_t S_, const arc_swiglu_block* blk, int32_t T, Low low_step,
+                         void* workspace, size_t ws_bytes, arc_stream_t stream) {
+  if (!h_bf16 || !blk || !blk->sublayers || blk->n_sublayers <= 0 || S_ <= 0 || T < 0) return ARC_ERR_INVALID_ARG;
   const int64_t d = blk->d, F = blk->ffn;
   if (d <= 0 || F <= 0 || d % 16 || F % 16) return ARC_ERR_INVALID_ARG;
   const size_t need = arc_recurrent_workspace_bytes(S_, blk);
@@ -570,7 +572,7 @@ arc_status arc_recurrent_prefill(void* h_bf16, int64_t S_, const arc_swiglu_bloc
   const size_t qws_bytes = ws_bytes - off[6];
   arc_status st;
   for (int32_t t = 0; t < T; ++t) {
-    const bool low = t < k_low;
+    const bool low = low_step(t);
     for (int i = 0; i < blk->n_sublayers; ++i) {
       const arc_swiglu_sublayer& L = blk->sublayers[i];
       if (low) {
@@ -598,6 +600,21 @@ arc_status arc_recurrent_prefill(void* h_bf16, int64_t S_, const arc_swiglu_bloc
     }
   }
   return ARC_OK;
+}
+}  // extern "C++"
+
+arc_status arc_recurrent_prefill(void* h_bf16, int64_t S_, const arc_swiglu_block* blk, int32_t T, int32_t k_low,
+                                 void* workspace, size_t ws_bytes, arc_stream_t stream) {
+  if (k_low < 0) return ARC_ERR_INVALID_ARG;
+  return recurrent_run(h_bf16, S_, blk, T, [k_low](int32_t t) { return t < k_low; }, workspace, ws_bytes, stream);
+}
+
+arc_status arc_recurrent_prefill_schedule(void* h_bf16, int64_t S_, const arc_swiglu_block* blk, int32_t T,
+                                          const uint8_t* low_steps, void* workspace, size_t ws_bytes,
+                                          arc_stream_t stream) {
+  if (T > 0 && !low_steps) return ARC_ERR_INVALID_ARG;
+  return recurrent_run(h_bf16, S_, blk, T, [low_steps](int32_t t) { return low_steps[t] != 0; }, workspace,
+                       ws_bytes, stream);
 }
 
 arc_status arc_last_device_status(arc_stream_t stream) {

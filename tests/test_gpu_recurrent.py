@@ -160,3 +160,24 @@ def test_ramp_schedule_error_ordering():
         errs[k] = (torch.linalg.norm(out - ref) / torch.linalg.norm(ref)).item()
     assert errs[0] == 0.0
     assert 0.0 < errs[4] < errs[8]
+
+
+@pytest.mark.parametrize("schedule", [[0, 1, 0, 1], [1, 1, 0, 0], [0, 0, 1, 1], [1, 0, 0, 1]])
+def test_schedule_driver_equals_composed_steps(schedule):
+    # any per-step precision schedule is the composition of its steps, each run on its own
+    # (one step of the prefix driver: k_low = 1 for an NVFP4 step, 0 for a BF16 one)
+    rec, h0, subs = make_block(S=130, d=256, ffn=512, r=32)
+    blk = arc.RecurrentBlock(256, 512, EPS, [{k: v for k, v in s.items() if k != "bits"} for s in subs])
+    h_drv = arc.recurrent_prefill_schedule(h0.clone(), blk, schedule)
+    h = h0.clone()
+    for f in schedule:
+        arc.recurrent_prefill(h, blk, 1, 1 if f else 0)
+    torch.cuda.synchronize()
+    assert arc.last_device_status() == 0
+    assert torch.equal(h_drv, h)
+    # the prefix schedule is the k_low driver
+    k = 2
+    a = arc.recurrent_prefill_schedule(h0.clone(), blk, [1] * k + [0] * 2)
+    b = arc.recurrent_prefill(h0.clone(), blk, 4, k)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
