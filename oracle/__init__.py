@@ -83,6 +83,9 @@ def lib():
                 "oracle_silu_mul_rows": (None, [P, I64, I64, P, I64, I64, I64]),
                 "oracle_e2m1_encode_array": (None, [P, I64, P]),
                 "oracle_e4m3_encode_array": (None, [P, I64, P]),
+                "oracle_fp8_scale": (F, [F]),
+                "oracle_e4m3_encode_signed": (ctypes.c_uint8, [F]),
+                "oracle_quantize_fp8_rows": (None, [P, I64, I64, F, P, I64, I64, I64]),
                 "oracle_e4m3_decode_array": (None, [P, I64, P]),
                 "oracle_e2m1_decode_array": (None, [P, I64, P]),
                 "oracle_e2m1_of_quotient_array": (None, [P, I64, F, P]),
@@ -304,6 +307,40 @@ def pack_weight_reordered(w, perm, r: int, s_w: float):
     perm = np.ascontiguousarray(np.asarray(perm, dtype=np.int64).reshape(-1))
     assert perm.size == w.shape[1] and 0 <= r <= perm.size
     return pack_weight(np.ascontiguousarray(w[:, perm]), np.arange(r, dtype=np.int32), s_w)
+
+
+def fp8_scale(amax_value: float) -> float:
+    """Per-tensor FP8 scale amax / 448 with the all-zero guard (arc_oracle.c, FP8 W8A8)."""
+    return float(lib().oracle_fp8_scale(float(np.float32(amax_value))))
+
+
+def e4m3_encode_signed(v) -> np.ndarray:
+    v = np.ascontiguousarray(np.asarray(v, dtype=np.float32)).reshape(-1)
+    L = lib()
+    return np.array([L.oracle_e4m3_encode_signed(float(t)) for t in v], np.uint8)
+
+
+def quantize_fp8(x, s: float) -> np.ndarray:
+    """X [M, K] bf16 -> E4M3 codes [M, K] of x / s (RAMP's FP8 weights and activations with one
+    per-tensor scale; arc_oracle.c, FP8 W8A8)."""
+    x = as_u16(x)
+    M, K = x.shape
+    codes = np.zeros((M, K), np.uint8)
+    L = lib()
+
+    def run(r0, r1):
+        L.oracle_quantize_fp8_rows(_ptr(x), K, K, float(np.float32(s)), _ptr(codes), K, r0, r1)
+
+    _split_rows(M, run, min_rows=16)
+    return codes
+
+
+def gemm_fp8_f64(a_codes, s_a: float, b_codes, s_b: float, rows=None) -> np.ndarray:
+    """Y = (s_a s_b) * E4M3(A) E4M3(B)^T in FP64 (a library matmul of the decoded operands)."""
+    a = np.ascontiguousarray(a_codes if rows is None else a_codes[rows])
+    A = e4m3_decode(a).astype(np.float64)
+    B = e4m3_decode(np.ascontiguousarray(b_codes)).astype(np.float64)
+    return (float(np.float32(s_a)) * float(np.float32(s_b))) * (A @ B.T)
 
 
 def dequant(codes, sf) -> np.ndarray:

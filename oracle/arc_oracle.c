@@ -507,6 +507,26 @@ void oracle_e4m3_encode_array(const float* v, int64_t n, uint8_t* out) {
   for (int64_t i = 0; i < n; ++i) out[i] = oracle_e4m3_encode_nonneg(v[i]);
 }
 
+/* ------------------------------------------------------------------------------------------ */
+/* FP8 W8A8 with per-tensor scales (the low-precision format of RAMP's own instantiation,        */
+/* "RAMP" §4.1: FP8 weights and activations): s = amax / 448 (the largest E4M3 magnitude), the  */
+/* all-zero guard s = 1, code = signed E4M3 of the fp32 quotient x / s (ties to even, saturating */
+/* at 448, the sign kept on values that round to zero, as for the E2M1 codes).                   */
+/* ------------------------------------------------------------------------------------------ */
+
+float oracle_fp8_scale(float amax) { return amax > 0.0f ? amax / 448.0f : 1.0f; }
+
+uint8_t oracle_e4m3_encode_signed(float v) {
+  const uint8_t mag = oracle_e4m3_encode_nonneg(fabsf(v));
+  return (uint8_t)((signbit(v) ? 0x80 : 0x00) | mag);
+}
+
+void oracle_quantize_fp8_rows(const uint16_t* x, int64_t K, int64_t ldx, float s, uint8_t* codes, int64_t ldc,
+                              int64_t m0, int64_t m1) {
+  for (int64_t m = m0; m < m1; ++m)
+    for (int64_t k = 0; k < K; ++k) codes[m * ldc + k] = oracle_e4m3_encode_signed(bf16_to_f32(x[m * ldx + k]) / s);
+}
+
 void oracle_e4m3_decode_array(const uint8_t* c, int64_t n, float* out) {
   for (int64_t i = 0; i < n; ++i) out[i] = oracle_e4m3_decode(c[i]);
 }
