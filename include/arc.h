@@ -212,6 +212,32 @@ arc_status arc_gemm_bf16(const void* x_bf16, int64_t ldx, const void* w_bf16, in
                          arc_stream_t stream);
 
 /* ----------------------------------------------------------------------------------------- */
+/* FP8 W8A8 ("RAMP…" §4.1: the low-precision steps run with FP8 weights and activations)        */
+/* ----------------------------------------------------------------------------------------- */
+
+/*
+ * Quantize X [M, K] bf16 (leading dimension ldx) to E4M3 codes [M, K] (leading dimension ldc
+ * bytes) with one per-tensor scale: s = amax(|x|)/448 (1 for an all-zero tensor), or
+ * *d_static_scale; code = signed E4M3 of the correctly rounded fp32 quotient x / s (ties to
+ * even, saturating at 448, the sign kept on a quotient that rounds to zero). The scale used is
+ * written to d_scale_out. Workspace: arc_quantize_workspace_bytes(M, 0) bytes, 256-byte aligned.
+ * Requires K % 16 == 0, ldx >= K with rows 16-byte aligned, ldc >= K, ldc % 16 == 0.
+ */
+arc_status arc_quantize_fp8(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, const float* d_static_scale,
+                            uint8_t* codes, int64_t ldc, float* d_scale_out, void* workspace, size_t ws_bytes,
+                            arc_stream_t stream);
+
+/*
+ * Y [M, N] bf16 = bf16_rn( (s_A * s_B) * sum_k E4M3(a) E4M3(b) [+ add] ) with A [M, K] and
+ * B [N, K] E4M3 codes (leading dimensions lda, ldb bytes), fp32 tensor-core accumulation
+ * (tcgen05 kind::f8f6f4). Requires K % 16 == 0, lda, ldb multiples of 16, N % 8 == 0,
+ * ldy % 8 == 0, 16-byte aligned pointers; add may alias y.
+ */
+arc_status arc_gemm_fp8(const uint8_t* a_codes, int64_t lda, const float* d_a_scale, const uint8_t* b_codes,
+                        int64_t ldb, const float* d_b_scale, int64_t M, int64_t N, int64_t K, void* y_bf16,
+                        int64_t ldy, const void* add_bf16, int64_t ld_add, arc_stream_t stream);
+
+/* ----------------------------------------------------------------------------------------- */
 /* Elementwise pieces of the recurrent SwiGLU block                                            */
 /* ----------------------------------------------------------------------------------------- */
 

@@ -92,6 +92,13 @@ _SIGS = {
                                                       ctypes.POINTER(SwigluBlock), ctypes.c_int32,
                                                       ctypes.POINTER(ctypes.c_uint8), ctypes.c_void_p,
                                                       ctypes.c_size_t, ctypes.c_void_p]),
+    "arc_quantize_fp8": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                        ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "arc_gemm_fp8": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                                    ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                    ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                    ctypes.c_int64, ctypes.c_void_p]),
     "arc_last_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "arc_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64]),
     "arc_debug_inject": (ctypes.c_int, [ctypes.c_int32]),
@@ -369,6 +376,44 @@ def recurrent_prefill_schedule(h: torch.Tensor, block: RecurrentBlock, schedule,
         _p(h), S, ctypes.byref(block.block), len(schedule), flags, _p(workspace), workspace.numel(),
         _stream(stream)))
     return h
+
+
+class FP8Tensor:
+    """E4M3 codes [rows, K] (row stride K bytes) and the device fp32 tensor scale."""
+
+    def __init__(self, codes: torch.Tensor, scale: torch.Tensor):
+        self.codes, self.scale = codes, scale
+        self.rows, self.k = codes.shape
+
+
+def quantize_fp8(x: torch.Tensor, static_scale: torch.Tensor | None = None, out: FP8Tensor | None = None,
+                 workspace: torch.Tensor | None = None, stream=None) -> FP8Tensor:
+    """arc_quantize_fp8: X [M, K] bf16 -> E4M3 codes with one per-tensor scale (amax/448)."""
+    _need_cuda(x, static_scale)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    M, K = x.shape
+    if out is None:
+        out = FP8Tensor(torch.empty(M, K, dtype=torch.uint8, device=x.device),
+                        torch.empty(1, dtype=torch.float32, device=x.device))
+    if workspace is None:
+        workspace = _ws(quantize_workspace_bytes(M, 0), x.device)
+    _check("arc_quantize_fp8", lib().arc_quantize_fp8(_p(x), M, K, x.stride(0), _p(static_scale), _p(out.codes),
+                                                      out.codes.stride(0), _p(out.scale), _p(workspace),
+                                                      workspace.numel(), _stream(stream)))
+    return out
+
+
+def gemm_fp8(a: FP8Tensor, b: FP8Tensor, out: torch.Tensor | None = None, add: torch.Tensor | None = None,
+             stream=None) -> torch.Tensor:
+    """arc_gemm_fp8: Y [M, N] bf16 = s_A s_B * E4M3(A) E4M3(B)^T (+ add)."""
+    assert a.k == b.k
+    M, N, K = a.rows, b.rows, a.k
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=a.codes.device)
+    _check("arc_gemm_fp8", lib().arc_gemm_fp8(
+        _p(a.codes), a.codes.stride(0), _p(a.scale), _p(b.codes), b.codes.stride(0), _p(b.scale), M, N, K,
+        _p(out), out.stride(0), _p(add), 0 if add is None else add.stride(0), _stream(stream)))
+    return out
 
 
 def last_device_status(stream=None) -> int:

@@ -1,12 +1,14 @@
 // gemm.cuh -- the compute-bound half of the hot path: one persistent, warp-specialised
-// tcgen05 GEMM skeleton instantiated twice.
-//   FP4 = true:  block-scaled NVFP4 GEMM of depth K_aug (tcgen05.mma kind::mxf4nvf4,
+// tcgen05 GEMM skeleton instantiated for three operand kinds.
+//   FP4:         block-scaled NVFP4 GEMM of depth K_aug (tcgen05.mma kind::mxf4nvf4,
 //                scale_vec::4X: one E4M3 scale per 16 elements of A and of B), the unified
 //                GEMM of "ARCQuant ... Augmented Residual Channels" (Unified GEMM Executie:
 //                one GEMM over K_in + S absorbs the residual correction by linearity), epilogue
 //                Y = bf16(s_A s_B acc [+ add]).
-//   FP4 = false: BF16 GEMM (tcgen05.mma kind::f16), the reference-precision switch of RAMP
+//   BF16:        BF16 GEMM (tcgen05.mma kind::f16), the reference-precision switch of RAMP
 //                (section 4.1: the recurrent steps after the switch run in BF16).
+//   FP8:         E4M3 x E4M3 GEMM (tcgen05.mma kind::f8f6f4) with per-tensor scales, epilogue
+//                Y = bf16(s_A s_B acc [+ add]): RAMP's own low-precision format (FP8 W8A8).
 //
 // CTA = 15 warps, one CTA per SM, persistent over 128 x 256 output tiles (grouped raster):
 //   warp 0       TMA producer: per stage an A tile of 128 rows x 128 bytes and a B tile of 256
@@ -43,11 +45,14 @@
 
 namespace arc {
 
-template <bool FP4>
+// GEMM kinds: the BF16 reference GEMM, the block-scaled NVFP4 GEMM, the per-tensor-scaled FP8 GEMM.
+constexpr int kGemmBF16 = 0, kGemmFP4 = 1, kGemmFP8 = 2;
+
+template <int KIND>
 struct GemmTraits;
 
 template <>
-struct GemmTraits<true> {
+struct GemmTraits<kGemmFP4> {
   static constexpr int BM = 128, BN = 256, STAGES = 4, ACC_STAGES = 1;
   static constexpr int A_BYTES = BM * 128, B_BYTES = BN * 128;
   static constexpr int SFA_BYTES = 4 * 512, SFB_BYTES = 2 * 4 * 512;
@@ -58,7 +63,7 @@ struct GemmTraits<true> {
 };
 
 template <>
-struct GemmTraits<false> {
+struct GemmTraits<kGemmBF16> {
   static constexpr int BM = 128, BN = 256, STAGES = 4, ACC_STAGES = 2;
   static constexpr int A_BYTES = BM * 128, B_BYTES = BN * 128;
   static constexpr int SFA_BYTES = 0, SFB_BYTES = 0;
@@ -68,12 +73,24 @@ struct GemmTraits<false> {
   static constexpr int SF_COL0 = 0, SF_SET_COLS = 0;
 };
 
+// FP8: the BF16 geometry (128 bytes of K per row and stage = 128 E4M3 values, 4 MMAs of K = 32)
+template <>
+struct GemmTraits<kGemmFP8> {
+  static constexpr int BM = 128, BN = 256, STAGES = 4, ACC_STAGES = 2;
+  static constexpr int A_BYTES = BM * 128, B_BYTES = BN * 128;
+  static constexpr int SFA_BYTES = 0, SFB_BYTES = 0;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t IDESC = idesc_f8(BM, BN);
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int SF_COL0 = 0, SF_SET_COLS = 0;
+};
+
 // Output staging for the TMA-store epilogue: per epilogue warp one 32-row x 16-column bf16 chunk.
 constexpr int kEpiStageBytes = 32 * 16 * 2;
 
-template <bool FP4>
+template <int KIND>
 constexpr int gemm_smem_bytes() {
-  return GemmTraits<FP4>::STAGES * GemmTraits<FP4>::STAGE_BYTES + 8 * kEpiStageBytes + 1024 + 256;
+  return GemmTraits<KIND>::STAGES * GemmTraits<KIND>::STAGE_BYTES + 8 * kEpiStageBytes + 1024 + 256;
 }
 
 // TMA tensor store of a box from shared memory (bulk-group completion), and its waits.
@@ -133,11 +150,12 @@ __device__ __forceinline__ uint4 lds_u32x4(uint32_t addr) {
 constexpr int kGemmThreads = 480;  // producer, 2 MMA issuers, 4 scale writers, 8 epilogue warps
 constexpr int kGemmEpiWarp0 = 7;
 
-template <bool FP4, bool ADD>
+template <int KIND, bool ADD>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
            const __grid_constant__ CUtensorMap tmY, const GemmArgs g) {
-  using T = GemmTraits<FP4>;
+  using T = GemmTraits<KIND>;
+  constexpr bool FP4 = KIND == kGemmFP4, FP8 = KIND == kGemmFP8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + T::STAGES * T::STAGE_BYTES;  // 8 x 1 KB, one per epilogue warp
@@ -205,7 +223,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               bytes += static_cast<uint32_t>(natoms * 512 * (1 + nb));
             }
             mbar_arrive_expect_tx(&full[stage], bytes);
-            const int kx = FP4 ? ks * 128 : ks * 64;
+            const int kx = (FP4 || FP8) ? ks * 128 : ks * 64;  // byte maps for FP4 / FP8, bf16 map
             tma_load_2d(sA, &tmA, &full[stage], kx, tm * T::BM);
             tma_load_2d(sB, &tmB, &full[stage], kx, tn * T::BN);
             if (FP4) {
@@ -250,7 +268,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_after();
           uint8_t* sA = smem + stage * T::STAGE_BYTES;
           uint8_t* sB = sA + T::A_BYTES;
-          const int nk = FP4 ? min(4, g.ksteps - 4 * ks) : 4;
+          const int nk = (FP4 || FP8) ? min(4, g.ksteps - 4 * ks) : 4;
           const uint64_t da = desc_kmajor_sw128(smem_u32(sA));
           const uint64_t db = desc_kmajor_sw128(smem_u32(sB));
           const uint32_t sf = tmem + T::SF_COL0 + T::SF_SET_COLS * stage;
@@ -259,6 +277,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t accum = (ks > 0 || k > 0) ? 1u : 0u;
             if (FP4)
               tc_mma_nvf4(d_tmem, da + off, db + off, T::IDESC, sf + 32 + 4 * k, sf + 8 * k, accum);
+            else if (FP8)
+              tc_mma_f8(d_tmem, da + off, db + off, T::IDESC, accum);
             else
               tc_mma_bf16(d_tmem, da + off, db + off, T::IDESC, accum);
           }
@@ -337,7 +357,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // stored 32 columns at a time.
     const int q = warp & 3;
     const int half = (warp - kGemmEpiWarp0) >> 2;
-    const float alpha = FP4 ? __fmul_rn(*g.a_scale, *g.b_scale) : 1.0f;
+    const float alpha = (FP4 || FP8) ? __fmul_rn(*g.a_scale, *g.b_scale) : 1.0f;
     const uint64_t alpha2 = f2_pack(alpha, alpha);
     constexpr int HB = T::BN / 2;  // columns per warp
     uint32_t acc = 0, acc_phase = 0;

@@ -48,14 +48,18 @@ arc_status device_check(int* sms) {
     d.ok = true;
   }
   if (!d.attrs_set) {
-    if (cudaFuncSetAttribute(arc::k_gemm<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             arc::gemm_smem_bytes<true>()) != cudaSuccess ||
-        cudaFuncSetAttribute(arc::k_gemm<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             arc::gemm_smem_bytes<true>()) != cudaSuccess ||
-        cudaFuncSetAttribute(arc::k_gemm<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             arc::gemm_smem_bytes<false>()) != cudaSuccess ||
-        cudaFuncSetAttribute(arc::k_gemm<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             arc::gemm_smem_bytes<false>()) != cudaSuccess ||
+    if (cudaFuncSetAttribute(arc::k_gemm<arc::kGemmFP4, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             arc::gemm_smem_bytes<arc::kGemmFP4>()) != cudaSuccess ||
+        cudaFuncSetAttribute(arc::k_gemm<arc::kGemmFP4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             arc::gemm_smem_bytes<arc::kGemmFP4>()) != cudaSuccess ||
+        cudaFuncSetAttribute(arc::k_gemm<arc::kGemmBF16, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             arc::gemm_smem_bytes<arc::kGemmBF16>()) != cudaSuccess ||
+        cudaFuncSetAttribute(arc::k_gemm<arc::kGemmBF16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             arc::gemm_smem_bytes<arc::kGemmBF16>()) != cudaSuccess ||
+        cudaFuncSetAttribute(arc::k_gemm<arc::kGemmFP8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             arc::gemm_smem_bytes<arc::kGemmFP8>()) != cudaSuccess ||
+        cudaFuncSetAttribute(arc::k_gemm<arc::kGemmFP8, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             arc::gemm_smem_bytes<arc::kGemmFP8>()) != cudaSuccess ||
         cudaFuncSetAttribute(arc::k_quant_rows<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              arc::kQRowsSmemMax) != cudaSuccess ||
         cudaFuncSetAttribute(arc::k_quant_rows<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -263,21 +267,21 @@ arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, con
 // GEMM driver
 // ---------------------------------------------------------------------------------------------
 
-template <bool FP4>
+template <int KIND>
 arc_status gemm_launch(const CUtensorMap& ta, const CUtensorMap& tb, GemmArgs g, int sms, bool add,
                        cudaStream_t s) {
   const int ntiles = g.tiles_m * g.tiles_n;
   const unsigned grid = static_cast<unsigned>(std::min(ntiles, sms));
-  const int smem = arc::gemm_smem_bytes<FP4>();
+  const int smem = arc::gemm_smem_bytes<KIND>();
   CUtensorMap ty;
   std::memset(&ty, 0, sizeof(ty));
   if (!add && !make_store_map(&ty, g.y, static_cast<uint64_t>(g.N), static_cast<uint64_t>(g.M),
                               static_cast<uint64_t>(g.ldy) * 2))
     return ARC_ERR_CUDA;
   if (add)
-    arc::k_gemm<FP4, true><<<grid, arc::kGemmThreads, smem, s>>>(ta, tb, ty, g);
+    arc::k_gemm<KIND, true><<<grid, arc::kGemmThreads, smem, s>>>(ta, tb, ty, g);
   else
-    arc::k_gemm<FP4, false><<<grid, arc::kGemmThreads, smem, s>>>(ta, tb, ty, g);
+    arc::k_gemm<KIND, false><<<grid, arc::kGemmThreads, smem, s>>>(ta, tb, ty, g);
   return launch_status();
 }
 
@@ -447,7 +451,7 @@ arc_status arc_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_sf, const flo
                 static_cast<uint64_t>(N), static_cast<uint64_t>(kpad / 2), 128, g.box_rows_b))
     return ARC_ERR_CUDA;
   g.inject = take_inject();
-  return gemm_launch<true>(ta, tb, g, sms, add_bf16 != nullptr, S(stream));
+  return gemm_launch<arc::kGemmFP4>(ta, tb, g, sms, add_bf16 != nullptr, S(stream));
 }
 
 arc_status arc_gemm_bf16(const void* x_bf16, int64_t ldx, const void* w_bf16, int64_t ldw, int64_t M, int64_t N,
@@ -484,7 +488,86 @@ arc_status arc_gemm_bf16(const void* x_bf16, int64_t ldx, const void* w_bf16, in
                 static_cast<uint64_t>(ldw * 2), 64, g.box_rows_b))
     return ARC_ERR_CUDA;
   g.inject = take_inject();
-  return gemm_launch<false>(ta, tb, g, sms, add_bf16 != nullptr, S(stream));
+  return gemm_launch<arc::kGemmBF16>(ta, tb, g, sms, add_bf16 != nullptr, S(stream));
+}
+
+arc_status arc_quantize_fp8(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, const float* d_static_scale,
+                            uint8_t* codes, int64_t ldc, float* d_scale_out, void* workspace, size_t ws_bytes,
+                            arc_stream_t stream) {
+  if (!x_bf16 || !codes || !d_scale_out) return ARC_ERR_INVALID_ARG;
+  if (M <= 0 || K <= 0 || K % 16 || ldx < K || ldc < K) return ARC_ERR_INVALID_ARG;
+  if (M > (1ll << 30) || K > (1ll << 24)) return ARC_ERR_UNSUPPORTED;
+  if (!al16(x_bf16) || (ldx * 2) % 16 || !al16(codes) || ldc % 16) return ARC_ERR_ALIGNMENT;
+  if (!workspace || ws_bytes < arc_quantize_workspace_bytes(M, 0)) return ARC_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ARC_ERR_ALIGNMENT;
+  int sms = 0;
+  arc_status st = device_check(&sms);
+  if (st != ARC_OK) return st;
+  cudaStream_t s = S(stream);
+  QuantWs w = carve_quant_ws(workspace);
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x_bf16);
+  int npartials = 0;
+  if (!d_static_scale) {
+    const int64_t items = M * ((K + arc::kAmaxSeg - 1) / arc::kAmaxSeg);
+    npartials = static_cast<int>(std::max<int64_t>(
+        1, std::min<int64_t>({(items + 7) / 8, static_cast<int64_t>(sms) * 4, arc::kMaxPartials})));
+    arc::k_amax<<<static_cast<unsigned>(npartials), 256, 0, s>>>(xb, ldx, static_cast<int>(M), static_cast<int>(K),
+                                                                w.partials);
+    if ((st = launch_status()) != ARC_OK) return st;
+  }
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(M, static_cast<int64_t>(sms) * 8)));
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cfg.attrs = pdl;
+  cfg.numAttrs = d_static_scale ? 0 : 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, arc::k_quant_fp8, xb, ldx, static_cast<int>(M), static_cast<int>(K),
+                                           d_static_scale, static_cast<const uint32_t*>(w.partials), npartials,
+                                           d_scale_out, codes, ldc);
+  return e == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
+}
+
+arc_status arc_gemm_fp8(const uint8_t* a_codes, int64_t lda, const float* d_a_scale, const uint8_t* b_codes,
+                        int64_t ldb, const float* d_b_scale, int64_t M, int64_t N, int64_t K, void* y_bf16,
+                        int64_t ldy, const void* add_bf16, int64_t ld_add, arc_stream_t stream) {
+  if (!a_codes || !b_codes || !d_a_scale || !d_b_scale || !y_bf16) return ARC_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0 || K % 16 || N % 8 || lda < K || ldb < K || ldy < N || ldy % 8)
+    return ARC_ERR_INVALID_ARG;
+  if (add_bf16 && (ld_add < N || ld_add % 8)) return ARC_ERR_INVALID_ARG;
+  if (M > (1ll << 30) || N > (1ll << 30) || K > (1ll << 24)) return ARC_ERR_UNSUPPORTED;
+  if (!al16(a_codes) || !al16(b_codes) || lda % 16 || ldb % 16 || !al16(y_bf16) || (add_bf16 && !al16(add_bf16)))
+    return ARC_ERR_ALIGNMENT;
+  int sms = 0;
+  arc_status st = device_check(&sms);
+  if (st != ARC_OK) return st;
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  g.M = static_cast<int>(M);
+  g.N = static_cast<int>(N);
+  g.ksteps = static_cast<int>((K + 31) / 32);  // one MMA per 32 values; the map zero-fills past K
+  g.kstages = (g.ksteps + 3) / 4;
+  g.tiles_m = static_cast<int>((M + 127) / 128);
+  g.tiles_n = static_cast<int>((N + 255) / 256);
+  g.box_rows_a = static_cast<int>(std::min<int64_t>(128, M));
+  g.box_rows_b = static_cast<int>(std::min<int64_t>(256, N));
+  g.a_scale = d_a_scale;
+  g.b_scale = d_b_scale;
+  g.y = static_cast<__nv_bfloat16*>(y_bf16);
+  g.ldy = ldy;
+  g.add = static_cast<const __nv_bfloat16*>(add_bf16);
+  g.ld_add = ld_add;
+  g.wait_ns = g_wait_ns;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                static_cast<uint64_t>(lda), 128, g.box_rows_a) ||
+      !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b_codes, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                static_cast<uint64_t>(ldb), 128, g.box_rows_b))
+    return ARC_ERR_CUDA;
+  g.inject = take_inject();
+  return gemm_launch<arc::kGemmFP8>(ta, tb, g, sms, add_bf16 != nullptr, S(stream));
 }
 
 arc_status arc_rmsnorm_bf16(const void* h_bf16, int64_t S_, int64_t d, int64_t ldh, const void* gain_bf16, float eps,

@@ -806,4 +806,78 @@ __global__ void __launch_bounds__(kQReoThreads, 3) k_quant_reordered(QuantArgs a
   }
 }
 
+
+// ---------------------------------------------------------------------------------------------
+// FP8 W8A8 coding with a per-tensor scale (RAMP: FP8 weights and activations in the
+// low-precision steps): s = amax / 448 (the largest E4M3 magnitude; 1 for an all-zero tensor),
+// code = signed E4M3 of the correctly rounded fp32 quotient x / s (ties to even, saturating at
+// 448, the sign kept on a quotient that rounds to zero). Quotients are formed negated from
+// -RN(1/s) with one Markstein correction, as for the E2M1 codes, and the sign bits flipped back;
+// a plain IEEE divide is used when s is outside [2^-90, 2^90].
+// ---------------------------------------------------------------------------------------------
+
+// Two fp32 -> two E4M3 bytes (round to nearest even, saturating), `lo` in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2_rn_sat(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__global__ void __launch_bounds__(256) k_quant_fp8(const __nv_bfloat16* __restrict__ x, int64_t ldx, int M, int K,
+                                                   const float* static_scale, const uint32_t* partials,
+                                                   int npartials, float* scale_out, uint8_t* codes, int64_t ldc) {
+  pdl_wait();
+  float s;
+  {
+    __shared__ uint32_t red[32];
+    __shared__ float s_sh;
+    if (static_scale) {
+      s = *static_scale;
+    } else {
+      uint32_t mx = 0;
+      for (int i = threadIdx.x; i < npartials; i += blockDim.x) mx = max(mx, partials[i]);
+      mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+      if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+      __syncthreads();
+      uint32_t b = 0;
+      for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) b = max(b, red[i]);
+      const float am = __uint_as_float(b);
+      s = am > 0.0f ? __fdiv_rn(am, 448.0f) : 1.0f;
+    }
+    if (threadIdx.x == 0) s_sh = s;
+    __syncthreads();
+    s = s_sh;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = s;
+  const bool fast = in_safe_range(s);
+  const float nr = fast ? -__frcp_rn(s) : 0.0f;
+  const uint64_t nrcp2 = f2_pack(nr, nr), s2 = f2_pack(s, s);
+  const int chunks = K >> 3;  // 8 values (16 bytes of X, 8 bytes of codes) each
+  for (int m = blockIdx.x; m < M; m += gridDim.x) {
+    const __nv_bfloat16* row = x + static_cast<int64_t>(m) * ldx;
+    uint8_t* crow = codes + static_cast<int64_t>(m) * ldc;
+    for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+      const uint4 w = ld_nc_v4(row + 8 * c);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+      uint32_t out[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t b01, b23;
+        if (fast) {
+          float q0, q1, q2, q3;
+          f2_unpack(neg_div2_rn(f2_pack(bf16_lo(ws[2 * h]), bf16_hi(ws[2 * h])), s2, nrcp2), q0, q1);
+          f2_unpack(neg_div2_rn(f2_pack(bf16_lo(ws[2 * h + 1]), bf16_hi(ws[2 * h + 1])), s2, nrcp2), q2, q3);
+          b01 = e4m3x2_rn_sat(q0, q1) ^ 0x8080u;
+          b23 = e4m3x2_rn_sat(q2, q3) ^ 0x8080u;
+        } else {
+          b01 = e4m3x2_rn_sat(__fdiv_rn(bf16_lo(ws[2 * h]), s), __fdiv_rn(bf16_hi(ws[2 * h]), s));
+          b23 = e4m3x2_rn_sat(__fdiv_rn(bf16_lo(ws[2 * h + 1]), s), __fdiv_rn(bf16_hi(ws[2 * h + 1]), s));
+        }
+        out[h] = b01 | (b23 << 16);
+      }
+      *reinterpret_cast<uint2*>(crow + 8 * c) = make_uint2(out[0], out[1]);
+    }
+  }
+}
+
 }  // namespace arc
