@@ -100,7 +100,10 @@ def layer_flops(L):
 
 
 def layer_quant_bytes(L):
-    """Algorithmic bytes of the quantizer: read X once, write codes and scale bytes."""
+    """Algorithmic bytes of the quantizer: read X once, write codes and scale bytes (FP8: one
+    byte per value, no block scales)."""
+    if L.get("fp8"):
+        return 3 * L["M"] * L["K"]
     kp = kpad(L["K"] + L["r"])
     return 2 * L["M"] * L["K"] + L["M"] * kp // 2 + L["M"] * kp // 16
 
@@ -217,11 +220,15 @@ def run_layers(args, rank, world, device, layers, with_error=False):
 
     stream = torch.cuda.Stream(device=device)
     reorder = getattr(args, "reorder", False)
+    fp8 = getattr(args, "format", "nvfp4") == "fp8"
     xs_host, xs, idx, packed, qa, ys, wsp, errs = {}, {}, {}, {}, {}, {}, {}, {}
     rs = {L["name"]: L["r"] for L in layers}
 
     def quant(name, **kw):
-        # the step's quantizer: natural channel order with the outlier list, or the reordered one
+        # the step's quantizer: FP8, or NVFP4 in the natural channel order with the outlier list,
+        # or NVFP4 reordered
+        if fp8:
+            return arc.quantize_fp8(xs[name], stream=stream, **kw)
         if reorder:
             return arc.quantize_act_nvfp4_reordered(xs[name], idx[name], rs[name], stream=stream, **kw)
         return arc.quantize_act_nvfp4(xs[name], idx[name], stream=stream, **kw)
@@ -233,7 +240,10 @@ def run_layers(args, rank, world, device, layers, with_error=False):
             xs_host[name] = W.to_torch_bf16(d["x"])
             xs[name] = xs_host[name].to(device)
             w = W.to_torch_bf16(d["w"]).to(device)
-            if reorder:
+            if fp8:
+                idx[name] = None
+                packed[name] = arc.quantize_fp8(w, stream=stream)  # weights: their own tensor scale
+            elif reorder:
                 # idx holds the full calibration order; its first r channels are the outliers
                 idx[name] = arc.calibrate_order(xs[name], stream=stream)
                 packed[name] = arc.pack_weight_nvfp4_reordered(w, idx[name], r, stream=stream)
@@ -245,7 +255,7 @@ def run_layers(args, rank, world, device, layers, with_error=False):
             wsp[name] = torch.empty(arc.quantize_workspace_bytes(M, r), dtype=torch.uint8, device=device)
             if with_error:
                 # relative error of the NVFP4 + ARC output against the BF16 product of the inputs
-                y = arc.gemm_nvfp4(qa[name], packed[name], stream=stream).float()
+                y = (arc.gemm_fp8 if fp8 else arc.gemm_nvfp4)(qa[name], packed[name], stream=stream).float()
                 yb = arc.gemm_bf16(xs[name], w, stream=stream).float()
                 errs[name] = (torch.linalg.norm(y - yb) / torch.linalg.norm(yb)).item()
             del w
@@ -261,7 +271,7 @@ def run_layers(args, rank, world, device, layers, with_error=False):
             quant(name, out=qa[name], workspace=wsp[name])
             if e1 is not None:
                 e1.record(stream)
-            arc.gemm_nvfp4(qa[name], packed[name], out=ys[name], stream=stream)
+            (arc.gemm_fp8 if fp8 else arc.gemm_nvfp4)(qa[name], packed[name], out=ys[name], stream=stream)
             if e2 is not None:
                 e2.record(stream)
                 rec.append((e0, e1, e2))
@@ -318,7 +328,7 @@ def run_layers(args, rank, world, device, layers, with_error=False):
                 name = L["name"]
                 xs[name].copy_(xs_pin[name], non_blocking=True)
                 quant(name, out=qa[name], workspace=wsp[name])
-                arc.gemm_nvfp4(qa[name], packed[name], out=ys[name], stream=stream)
+                (arc.gemm_fp8 if fp8 else arc.gemm_nvfp4)(qa[name], packed[name], out=ys[name], stream=stream)
                 ys_pin[name].copy_(ys[name], non_blocking=True)
 
         with torch.cuda.stream(stream):
@@ -353,11 +363,14 @@ def layers_line(args, world, layers, desc, res):
     value = step_flops * world * args.steps / (res["total_ms"] * 1e-3) / 1e12
     achieved = step_flops * args.steps / (res["g_ms"] * 1e-3) / 1e12
     quant_gbs = qbytes * args.steps / (res["q_ms"] * 1e-3) / 1e9
-    peak = pk["bf16_tflops"] * FP4_OVER_BF16
+    fp8 = getattr(args, "format", "nvfp4") == "fp8"
+    ratio = 2.0 if fp8 else FP4_OVER_BF16  # nominal dense FP8 / BF16 = 2, FP4 / BF16 = 4
+    peak = pk["bf16_tflops"] * ratio
     return {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC if not fp8 else "FP8 W8A8 GEMM TFLOP/s (% FP8 peak) + act-quant GB/s, 1×B200", "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": res["total_ms"] / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "e2m1 x e2m1 -> f32 (bf16 out)",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 x e4m3 -> f32 (bf16 out)" if fp8 else "e2m1 x e2m1 -> f32 (bf16 out)",
         "data": "synthetic (seeded; random weights and activations of the stated shapes)",
         "config": {"workload": desc, "l2": "flushed (256 MiB write) before every step",
                    "parallelism": f"replicas x{world}",
@@ -365,17 +378,18 @@ def layers_line(args, world, layers, desc, res):
                    else "natural (outlier list)"},
         "quant_gbs": quant_gbs,
         "gemm_only_tflops": achieved,
-        "pct_fp4_peak": 100.0 * value / peak,
+        ("pct_fp8_peak" if fp8 else "pct_fp4_peak"): 100.0 * value / peak,
         "per_projection": res["per_layer"],
-        "roofline": {"bound": "tensor", "kernel": f"k_gemm<nvfp4> (all {len(layers)} launches of a step)",
+        "roofline": {"bound": "tensor",
+                     "kernel": f"k_gemm<{'fp8' if fp8 else 'nvfp4'}> (all {len(layers)} launches of a step)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_source": f"{src} bf16 burst {pk['bf16_tflops']} TFLOP/s x {FP4_OVER_BF16:g} "
-                                    f"(nominal FP4/BF16 dense ratio)",
+                     "peak_source": f"{src} bf16 burst {pk['bf16_tflops']} TFLOP/s x {ratio:g} "
+                                    f"(nominal {'FP8' if fp8 else 'FP4'}/BF16 dense ratio)",
                      "traffic": ncu_traffic() if args.workload == "llama8b" and not getattr(args, "reorder", False)
-                     else None},
+                     and not fp8 else None},
         "quant_roofline": {"bound": "hbm",
-                           "kernel": "k_amax + " + ("k_quant_reordered" if getattr(args, "reorder", False)
-                                                    else "k_quant_rows"),
+                           "kernel": "k_amax + " + ("k_quant_fp8" if fp8 else "k_quant_reordered"
+                                                    if getattr(args, "reorder", False) else "k_quant_rows"),
                            "achieved": quant_gbs,
                            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": quant_gbs / pk["hbm_gbs"],
                            "peak_source": f"{src} copy bandwidth"},
@@ -620,6 +634,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
     ap.add_argument("--proj", default="all", help="profiling: run only this layer (e.g. qkv, gateup)")
+    ap.add_argument("--format", default="nvfp4", choices=["nvfp4", "fp8"],
+                    help="linear-layer workloads: NVFP4 + ARC (default) or FP8 W8A8 with per-tensor scales")
     ap.add_argument("--reorder", action="store_true",
                     help="linear-layer workloads: channels reordered by calibration abs-max before the primary "
                          "quantization (the outlier set is the first r of the order)")
@@ -638,6 +654,11 @@ def main():
             if not layers:
                 ap.error("unknown --proj")
     if args.impl == "reference":
+        if args.format == "fp8":
+            if rank == 0:
+                print(json.dumps({"impl": "reference",
+                                  "unavailable": "the oracle arm times the NVFP4 + ARC format only"}))
+            return
         if layers is None:
             if rank == 0:
                 print(json.dumps({"impl": "reference",
@@ -655,10 +676,15 @@ def main():
         if args.workload == "recurrent":
             line = run_recurrent(args, rank, world, device)
         else:
+            if args.format == "fp8":
+                if args.reorder:
+                    ap.error("--reorder applies to the NVFP4 format")
+                for L in layers:
+                    L["r"], L["fp8"] = 0, True
             res = run_layers(args, rank, world, device, layers,
-                             with_error=args.workload == "stress" or args.reorder)
+                             with_error=args.workload == "stress" or args.reorder or args.format == "fp8")
             line = layers_line(args, world, layers, desc, res) if rank == 0 else None
-            if rank == 0 and not args.no_cpu_baseline:
+            if rank == 0 and not args.no_cpu_baseline and args.format != "fp8":
                 line["cpu_baseline"] = cpu_baseline(layers, reorder=args.reorder)
         if rank == 0:
             print(json.dumps(line), flush=True)
