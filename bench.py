@@ -77,7 +77,7 @@ def layer_set(workload: str):
             key = (frac, rows, row0)
             if key not in cache:
                 cache.clear()
-                cache[key] = W.stress(frac, rows=rows)
+                cache[key] = W.stress(frac, rows=rows, row0=row0)
             return cache[key]
 
         for frac in c["fracs"]:
@@ -208,6 +208,17 @@ def _ev():
 def _barrier(world):
     if world > 1:
         torch.distributed.barrier()
+
+
+def ranks_max(vals, device):
+    """Element-wise maximum over the ranks (a job's time is its slowest rank's); the values
+    themselves on one rank. Works with any process-group backend (NCCL on the GPUs, gloo in the
+    CPU tests)."""
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    if torch.distributed.is_available() and torch.distributed.is_initialized() and \
+            torch.distributed.get_world_size() > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
 
 
 # ---------------------------------------------------------------------------------------------
@@ -348,10 +359,7 @@ def run_layers(args, rank, world, device, layers, with_error=False):
         _barrier(world)
         e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
 
-    t = torch.tensor([total_ms, q_ms, g_ms, e2e_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    total_ms, q_ms, g_ms, e2e_ms = t.tolist()
+    total_ms, q_ms, g_ms, e2e_ms = ranks_max([total_ms, q_ms, g_ms, e2e_ms], device)
     return dict(total_ms=total_ms, q_ms=q_ms, g_ms=g_ms, e2e_ms=e2e_ms, per_layer=per_layer, clocks=clocks,
                 h2d=h2d, d2h=d2h, launches=args.steps * len(layers) * 3)
 
@@ -475,10 +483,7 @@ def run_recurrent(args, rank, world, device):
         raise RuntimeError("device status set during the timed prefills")
     for k, a, b in evs:
         times[k].append(a.elapsed_time(b))
-    t = torch.tensor([statistics.mean(times[k]) for k in k_lows], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms = dict(zip(k_lows, t.tolist()))
+    ms = dict(zip(k_lows, ranks_max([statistics.mean(times[k]) for k in k_lows], device)))
     per = {}
     for k in k_lows:
         fl = (k * f_fp4 + (T - k) * f_bf16) * world

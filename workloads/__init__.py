@@ -179,14 +179,14 @@ def llama8b(proj: str, rows: int | None = None, row0: int = 0, with_w: bool = Tr
     return dict(x=x, w=w, r=LLAMA8B_R, K=K, N=N, M=M, outliers=np.nonzero(mult != 1.0)[0])
 
 
-def stress(frac: float, rows: int | None = None, w_rows: int | None = None):
+def stress(frac: float, rows: int | None = None, w_rows: int | None = None, row0: int = 0):
     c = STRESS
     t = list(c["fracs"]).index(frac)
     K = c["K"]
     M = c["M"] if rows is None else rows
     n_out = int(round(frac * K))
     mult = outlier_multipliers(c["seed"], t, K, n_out, 10.0, 200.0)
-    x = matrix_bf16(c["seed"], stream_id(t, 1), M, K, 1.0, dist="t3", col_mult=mult)
+    x = matrix_bf16(c["seed"], stream_id(t, 1), M, K, 1.0, dist="t3", col_mult=mult, row0=row0)
     w = matrix_bf16(c["seed"], stream_id(0, 2), c["N"] if w_rows is None else w_rows, K, 0.02)
     return dict(x=x, w=w, K=K, N=c["N"], M=M, outliers=np.nonzero(mult != 1.0)[0])
 
