@@ -68,3 +68,32 @@ def test_host_checks_reject_before_any_launch(L):
     assert L.arc_gemm_bf16(P(0x10004), 64, fake, 64, 4, 16, 64, fake, 16, None, 0, None) == 2
     assert L.arc_set_wait_limit_ns(0) == 1
     assert L.arc_debug_inject(7) == 1
+
+
+def test_host_checks_of_the_reorder_fp8_and_schedule_calls(L):
+    P = ctypes.c_void_p
+    fake, ws = P(0x10000), P(0x20000)
+    # calibration order: odd K, NULL output, small workspace, misaligned input
+    assert L.arc_calibrate_order(fake, 4, 63, 64, fake, ws, 1 << 20, None) == 1
+    assert L.arc_calibrate_order(fake, 4, 64, 64, None, ws, 1 << 20, None) == 1
+    assert L.arc_calibrate_order(fake, 4, 64, 64, fake, ws, 8, None) == 6
+    assert L.arc_calibrate_order(P(0x10002), 4, 64, 64, fake, ws, 1 << 20, None) == 2
+    # reordered quantizer / packer: NULL order, rows too wide for the two row buffers, misaligned order
+    assert L.arc_quantize_act_nvfp4_reordered(fake, 4, 64, 64, None, 16, None, 1e-6, None, fake, fake, fake, ws,
+                                              1 << 20, None) == 1
+    assert L.arc_quantize_act_nvfp4_reordered(fake, 4, 51216, 51216, fake, 16, None, 1e-6, None, fake, fake, fake,
+                                              ws, 1 << 20, None) == 3
+    assert L.arc_quantize_act_nvfp4_reordered(fake, 4, 64, 64, P(0x10004), 16, None, 1e-6, None, fake, fake, fake,
+                                              ws, 1 << 20, None) == 2
+    assert L.arc_pack_weight_nvfp4_reordered(fake, 4, 64, 64, None, 16, fake, fake, fake, ws, 1 << 20, None) == 1
+    # FP8 quantizer: K % 16, ldc < K, ldc % 16, small workspace
+    assert L.arc_quantize_fp8(fake, 4, 40, 40, None, fake, 48, fake, ws, 1 << 20, None) == 1
+    assert L.arc_quantize_fp8(fake, 4, 64, 64, None, fake, 48, fake, ws, 1 << 20, None) == 1
+    assert L.arc_quantize_fp8(fake, 4, 64, 64, None, fake, 72, fake, ws, 1 << 20, None) == 2
+    assert L.arc_quantize_fp8(fake, 4, 64, 64, None, fake, 64, fake, ws, 8, None) == 6
+    # FP8 GEMM: K % 16, lda % 16, N % 8
+    assert L.arc_gemm_fp8(fake, 40, fake, fake, 40, fake, 4, 16, 40, fake, 16, None, 0, None) == 1
+    assert L.arc_gemm_fp8(fake, 72, fake, fake, 64, fake, 4, 16, 64, fake, 16, None, 0, None) == 2
+    assert L.arc_gemm_fp8(fake, 64, fake, fake, 64, fake, 4, 12, 64, fake, 16, None, 0, None) == 1
+    # schedule driver: T > 0 steps and no flags
+    assert L.arc_recurrent_prefill_schedule(fake, 16, None, 4, None, ws, 1 << 20, None) == 1
