@@ -1,5 +1,6 @@
-// quant.cuh -- the memory-bound half of the hot path: RMSNorm statistics and the single-launch
-// NVFP4 quantizer with its augmented residual channels.
+// quant.cuh -- the memory-bound half of the hot path: RMSNorm statistics, the NVFP4 quantizer
+// with its augmented residual channels (natural channel order or reordered), and the FP8
+// per-tensor quantizer.
 //
 // Method ("ARCQuant: Boosting NVFP4 Quantization with Augmented Residual Channels for LLMs",
 // Methodologie, Dual-Stage Quantisatie / Kernel Implementatie; "Day 0 LLM Inference Support",
@@ -19,8 +20,12 @@
 //                 CTA forms the residual (activations) or value (weights) of each outlier
 //                 channel from the blocks holding outliers, which the coding threads kept in
 //                 shared memory (values, codes, d), stages them in its stash, codes the r/16
-//                 appended blocks and zero-fills the padding up to K_pad. A row never leaves its warp, so no grid-wide
-//                 synchronisation is needed.
+//                 appended blocks and zero-fills the padding up to K_pad. A row never leaves its
+//                 CTA, so no grid-wide synchronisation is needed.
+//   k_quant_reordered  the same coding with the channels in calibration order: rows staged in
+//                 shared memory by 1-D bulk copies, each block gathered through the permutation,
+//                 appended block j formed from primary block j in registers.
+//   k_quant_fp8   FP8 W8A8: signed E4M3 codes of x / (amax / 448), one thread per 8 values.
 // Divisions are correctly rounded: x/d is formed as the negated quotient from -RN(1/d) with one
 // exact-remainder correction (Markstein), which keeps the sign of zero quotients, and the codes
 // of the negated quotients have their sign bits flipped back; a plain IEEE divide is used when
