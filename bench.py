@@ -45,6 +45,7 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 METRIC = "NVFP4 ARC GEMM TFLOP/s (% FP4 peak) + fused act-quant GB/s, 1×B200"
+METRIC_FP8 = "FP8 W8A8 GEMM TFLOP/s (% FP8 peak) + act-quant GB/s, 1×B200"
 UNIT = "TFLOP/s"
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLOP/s)
 
@@ -375,7 +376,7 @@ def layers_line(args, world, layers, desc, res):
     ratio = 2.0 if fp8 else FP4_OVER_BF16  # nominal dense FP8 / BF16 = 2, FP4 / BF16 = 4
     peak = pk["bf16_tflops"] * ratio
     return {
-        "metric": METRIC if not fp8 else "FP8 W8A8 GEMM TFLOP/s (% FP8 peak) + act-quant GB/s, 1×B200", "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC_FP8 if fp8 else METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": res["total_ms"] / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3 x e4m3 -> f32 (bf16 out)" if fp8 else "e2m1 x e2m1 -> f32 (bf16 out)",
@@ -549,13 +550,17 @@ def schedule_study(arc, h, h0, blk, wsp, flush, stream, T, budget, ref, device, 
 # Oracle arm (CPU)
 # ---------------------------------------------------------------------------------------------
 
-def oracle_cache(layers, n_rows: int, reorder: bool = False):
+def oracle_cache(layers, n_rows: int, reorder: bool = False, fp8: bool = False):
     import oracle as O
 
     cache = {}
     for L in layers:
         d = L["gen"](n_rows, 0)
         x = d["x"][:n_rows]
+        if fp8:
+            sa, sw = O.fp8_scale(O.amax(x)), O.fp8_scale(O.amax(d["w"]))
+            cache[L["name"]] = dict(x=x, sa=sa, sw=sw, bc=O.quantize_fp8(d["w"], sw), fp8=True)
+            continue
         sa = O.tensor_scale(O.amax(x))
         sw = O.tensor_scale(O.amax(d["w"]))
         if reorder:
@@ -564,7 +569,7 @@ def oracle_cache(layers, n_rows: int, reorder: bool = False):
         else:
             idx = O.calibrate(x, L["r"]) if L["r"] else np.zeros(0, np.int32)
             bc, bsf = O.pack_weight(d["w"], idx, sw)  # every output column needs the full weight
-        cache[L["name"]] = dict(x=x, idx=idx, sa=sa, sw=sw, bc=bc, bsf=bsf, reorder=reorder)
+        cache[L["name"]] = dict(x=x, idx=idx, sa=sa, sw=sw, bc=bc, bsf=bsf, reorder=reorder, fp8=False)
     return cache
 
 
@@ -577,6 +582,10 @@ def oracle_sample_step(layers, rows: int, cache: dict):
     flops = 0.0
     for L in layers:
         c = cache[L["name"]]
+        if c["fp8"]:
+            O.gemm_fp8_f64(O.quantize_fp8(c["x"][:rows], c["sa"]), c["sa"], c["bc"], c["sw"])
+            flops += 2.0 * rows * L["N"] * L["K"]
+            continue
         if c["reorder"]:
             ac, asf = O.quantize_act_reordered(c["x"][:rows], c["idx"], L["r"], c["sa"])
         else:
@@ -586,13 +595,13 @@ def oracle_sample_step(layers, rows: int, cache: dict):
     return flops
 
 
-def cpu_baseline(layers, rows: int | None = None, reorder: bool = False):
+def cpu_baseline(layers, rows: int | None = None, reorder: bool = False, fp8: bool = False):
     """The oracle on the host cores: `rows` token rows (default two per host thread, so every
     thread works) of each layer, about 10-30 s of CPU work."""
     import oracle as O
 
     rows = rows or 2 * O._threads()
-    cache = oracle_cache(layers, max(rows, 64), reorder)
+    cache = oracle_cache(layers, max(rows, 64), reorder, fp8)
     t0 = time.perf_counter()
     flops = oracle_sample_step(layers, rows, cache)
     dt = time.perf_counter() - t0
@@ -607,7 +616,7 @@ def run_reference(args, rank, world, layers, desc):
     import oracle as O
 
     rows = O._threads()  # one token row per host thread per step
-    cache = oracle_cache(layers, max(rows, 64), getattr(args, "reorder", False))
+    cache = oracle_cache(layers, max(rows, 64), getattr(args, "reorder", False), getattr(args, "format", "") == "fp8")
     for _ in range(args.warmup):
         oracle_sample_step(layers, rows, cache)
     t0 = time.perf_counter()
@@ -616,7 +625,8 @@ def run_reference(args, rank, world, layers, desc):
         flops += oracle_sample_step(layers, rows, cache)
     dt = time.perf_counter() - t0
     v = flops / dt / 1e12
-    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+    metric = METRIC_FP8 if getattr(args, "format", "") == "fp8" else METRIC
+    line = {"impl": "reference", "metric": metric, "value": v, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{desc} (oracle on a row sample)", "sample_rows_per_projection": rows},
@@ -658,12 +668,12 @@ def main():
             layers = [L for L in layers if L["name"] == args.proj]
             if not layers:
                 ap.error("unknown --proj")
+    if args.format == "fp8" and layers is not None:
+        if args.reorder:
+            ap.error("--reorder applies to the NVFP4 format")
+        for L in layers:
+            L["r"], L["fp8"] = 0, True
     if args.impl == "reference":
-        if args.format == "fp8":
-            if rank == 0:
-                print(json.dumps({"impl": "reference",
-                                  "unavailable": "the oracle arm times the NVFP4 + ARC format only"}))
-            return
         if layers is None:
             if rank == 0:
                 print(json.dumps({"impl": "reference",
@@ -681,16 +691,11 @@ def main():
         if args.workload == "recurrent":
             line = run_recurrent(args, rank, world, device)
         else:
-            if args.format == "fp8":
-                if args.reorder:
-                    ap.error("--reorder applies to the NVFP4 format")
-                for L in layers:
-                    L["r"], L["fp8"] = 0, True
             res = run_layers(args, rank, world, device, layers,
                              with_error=args.workload == "stress" or args.reorder or args.format == "fp8")
             line = layers_line(args, world, layers, desc, res) if rank == 0 else None
-            if rank == 0 and not args.no_cpu_baseline and args.format != "fp8":
-                line["cpu_baseline"] = cpu_baseline(layers, reorder=args.reorder)
+            if rank == 0 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline(layers, reorder=args.reorder, fp8=args.format == "fp8")
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:
