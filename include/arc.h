@@ -4,7 +4,8 @@
  * The method (sources by page title and section):
  *   "ARCQuant: Boosting NVFP4 Quantization with Augmented Residual Channels for LLMs"
  *     (Technische Samenvatting, Methodologie): NVFP4 blocks of 16 E2M1 values; outlier channels
- *     identified offline by calibration abs-max; primary block-wise quantization; the residual
+ *     identified offline by calibration abs-max (optionally all channels reordered by it before
+ *     the primary stage); primary block-wise quantization; the residual
  *     x - dequant(Q(x)) of the outlier channels quantized again as a second set of NVFP4
  *     channels and appended along K; the matching weight columns duplicated; one unified GEMM
  *     of depth K + r whose linear accumulation adds the correction; one fused kernel for
@@ -15,8 +16,9 @@
  *     producing operator, block-scaled tensor-core instructions consuming the scales directly.
  *   "RAMP: Recurrent Adaptive Mixed Precision for Efficient Prefill in Recurrent-Depth
  *     Language Models" (sections 2.1, 4.1, 4.2): a shared block applied T times; low-precision
- *     weight-and-activation steps before step k_low, reference-precision (BF16) steps after;
- *     hidden state kept in BF16.
+ *     weight-and-activation steps before step k_low (or on any schedule of steps),
+ *     reference-precision (BF16) steps after; hidden state kept in BF16; FP8 weights and
+ *     activations as the pages' own low-precision format.
  *
  * Number formats (the pages name E2M1 and block size 16; the rest is this library's reading):
  *   element   E2M1 code, 4 bits, magnitudes {0,.5,1,1.5,2,3,4,6}, bit 3 = sign
@@ -149,7 +151,7 @@ arc_status arc_calibrate_outliers(const void* x_bf16, int64_t M, int64_t K, int6
  * X [M, K] in descending abs-max order, ties by ascending index, written to d_perm_out (device
  * int32[K]); its first r entries are what arc_calibrate_outliers returns for r. Workspace as
  * arc_calibrate_outliers. The ranking does O(K^2) comparisons on the device (a calibration
- * step: about 0.1 ms at K = 28672). 0 < K <= 2^20, K even, x 4-byte aligned.
+ * step, run once per model). 0 < K <= 2^20, K even, x 4-byte aligned.
  */
 arc_status arc_calibrate_order(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, int32_t* d_perm_out,
                                void* workspace, size_t ws_bytes, arc_stream_t stream);
