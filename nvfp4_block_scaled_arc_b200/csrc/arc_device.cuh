@@ -29,16 +29,6 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Release store / acquire load at GPU scope (grid-level flags between CTAs).
-__device__ __forceinline__ void st_release_gpu(unsigned long long* p, unsigned long long v) {
-  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-__device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-
 // ---------------------------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------------------------
@@ -349,13 +339,5 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// E2M1 code of one fp32 value (round to nearest even, saturating, sign kept on zero).
-__device__ __forceinline__ uint32_t e2m1_rn_sat1(float q) {
-  uint16_t r;
-  asm("{\n\t.reg .b8 b0;\n\tcvt.rn.satfinite.e2m1x2.f32 b0, %1, %2;\n\tcvt.u16.u8 %0, b0;\n\t}"
-      : "=h"(r)
-      : "f"(0.0f), "f"(q));
-  return r & 0xFu;
-}
 
 }  // namespace arc

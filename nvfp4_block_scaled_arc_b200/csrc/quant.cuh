@@ -63,11 +63,6 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   return v;
 }
 
-__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
 
 __device__ __forceinline__ bool in_safe_range(float v) {
   return v >= 8.077935669463161e-28f && v <= 1.2379400392853803e27f;  // [2^-90, 2^90]
@@ -138,8 +133,12 @@ __device__ __forceinline__ uint32_t block_sf(float amax, float s, float rcp_s, f
   return e4m3_rn_sat(t);
 }
 
-// Codes of 16 values against decode scale d > 0 with nrcp = -RN(1/d) taken from a table (0 when
-// d is outside the range where the reciprocal form is exact): same result as encode16.
+// Codes of 16 values (8 packed pairs) against decode scale d > 0, with nrcp = -RN(1/d) taken from
+// a table (0 when d is outside [2^-90, 2^90], where the plain IEEE divide is used): E2M1 of the
+// correctly rounded quotient with the sign of x (a quotient that rounds to zero keeps it: -0.1 ->
+// 0x8). The quotients are formed negated, which keeps signed zeros exact, and since E2M1 is
+// sign-magnitude with symmetric rounding and saturation, code(q) = code(-q) ^ 8 nibble by nibble.
+// Element i of pair j in bits 8j + 4i.
 __device__ __forceinline__ uint2 encode16_nr(const uint64_t (&p)[8], float d, float nrcp) {
   if (nrcp == 0.0f) {
     float x[16];
@@ -158,33 +157,6 @@ __device__ __forceinline__ uint2 encode16_nr(const uint64_t (&p)[8], float d, fl
   return make_uint2(e2m1x8_rn_sat(lo) ^ 0x88888888u, e2m1x8_rn_sat(hi) ^ 0x88888888u);
 }
 
-// Codes of 16 values (8 packed pairs) against decode scale d > 0: E2M1 of the correctly rounded
-// quotient with the sign of x (a quotient that rounds to zero keeps it: -0.1 -> 0x8). The
-// quotients are formed negated, which keeps signed zeros exact, and since E2M1 is sign-magnitude
-// with symmetric rounding and saturation, code(q) = code(-q) ^ 8 nibble by nibble. Element i of
-// pair j in bits 8j + 4i.
-__device__ __forceinline__ uint2 encode16(const uint64_t (&p)[8], float d) {
-  if (!in_safe_range(d)) {
-    float x[16];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) f2_unpack(p[j], x[2 * j], x[2 * j + 1]);
-    // the hardware conversion keeps the sign of a zero quotient, like the negated fast path
-    return encode16_slow(d, x[0], x[1], x[2], x[3], x[4], x[5], x[6], x[7], x[8], x[9], x[10], x[11], x[12],
-                         x[13], x[14], x[15]);
-  }
-  float nq[16];
-  const float nrcp = -__frcp_rn(d);
-  const uint64_t nrcp2 = f2_pack(nrcp, nrcp), d2 = f2_pack(d, d);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) f2_unpack(neg_div2_rn(p[j], d2, nrcp2), nq[2 * j], nq[2 * j + 1]);
-  float lo[8], hi[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    lo[i] = nq[i];
-    hi[i] = nq[8 + i];
-  }
-  return make_uint2(e2m1x8_rn_sat(lo) ^ 0x88888888u, e2m1x8_rn_sat(hi) ^ 0x88888888u);
-}
 
 // RMSNorm of one bf16 value: bf16( fp32( (h * inv) * g ) ), products in double.
 __device__ __forceinline__ float rms_apply(float h, double inv, float g) {
