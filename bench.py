@@ -16,7 +16,15 @@ Other workloads (--workload), same timing rules:
   recurrent  the shared 2-sublayer SwiGLU block (d = 2048, ffn = 8192, RMSNorm, residual add)
              applied T = 16 times to H [4096, 2048]: one prefill per k_low in {0, 8, 12, 16}
              (steps before k_low in NVFP4 + ARC with r = 64, the rest BF16); time per prefill,
-             speedup against k_low = 0 and the hidden-state error against all-BF16
+             speedup against k_low = 0 and the hidden-state error against all-BF16; after the
+             timed region, a schedule study at 12 of 16 NVFP4 steps (RAMP's order, BF16 first,
+             interleaved, random placements): error and time of each
+
+Variants of the linear-layer workloads:
+  --reorder      channels reordered by calibration abs-max before the primary quantization
+                 (the outlier set is the first r of the order); adds the error against BF16
+  --format fp8   FP8 W8A8 with per-tensor scales instead of NVFP4 + ARC (metric: FP8 GEMM
+                 TFLOP/s against 2 x the measured BF16 peak); adds the error against BF16
 
 Metric: NVFP4 ARC GEMM TFLOP/s = sum over the step of 2*M*N*(K+r) / step time, with the fused
 activation quantizer's GB/s (read X + write codes + scale bytes) beside it.
