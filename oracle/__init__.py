@@ -84,6 +84,9 @@ def lib():
                 "oracle_e2m1_encode_array": (None, [P, I64, P]),
                 "oracle_e4m3_encode_array": (None, [P, I64, P]),
                 "oracle_fp8_scale": (F, [F]),
+                "oracle_mxfp4_scale_byte": (ctypes.c_uint8, [F]),
+                "oracle_quantize_mxfp4_rows": (None, [P, I64, I64, P, P, I64, I64]),
+                "oracle_gemm_mxfp4_f64": (None, [P, P, P, P, I64, I64, P, I64, P]),
                 "oracle_e4m3_encode_signed": (ctypes.c_uint8, [F]),
                 "oracle_quantize_fp8_rows": (None, [P, I64, I64, F, P, I64, I64, I64]),
                 "oracle_e4m3_decode_array": (None, [P, I64, P]),
@@ -341,6 +344,47 @@ def gemm_fp8_f64(a_codes, s_a: float, b_codes, s_b: float, rows=None) -> np.ndar
     A = e4m3_decode(a).astype(np.float64)
     B = e4m3_decode(np.ascontiguousarray(b_codes)).astype(np.float64)
     return (float(np.float32(s_a)) * float(np.float32(s_b))) * (A @ B.T)
+
+
+def mxfp4_scale_byte(amax_block: float) -> int:
+    """E8M0 scale byte of a 32-value MXFP4 block with abs-max amax_block (arc_oracle.c, MXFP4)."""
+    return int(lib().oracle_mxfp4_scale_byte(float(np.float32(amax_block))))
+
+
+def quantize_mxfp4(x):
+    """X [M, K] bf16 -> MXFP4 (OCP microscaling reading of ARCQuant's MXFP4 extension): codes
+    [M, K/2] (element k at byte k/2, low nibble for even k) and E8M0 scale bytes [M, K/32]."""
+    x = as_u16(x)
+    M, K = x.shape
+    assert K % 32 == 0
+    codes = np.zeros((M, K // 2), np.uint8)
+    scales = np.zeros((M, K // 32), np.uint8)
+    L = lib()
+
+    def run(r0, r1):
+        L.oracle_quantize_mxfp4_rows(_ptr(x), K, K, _ptr(codes), _ptr(scales), r0, r1)
+
+    _split_rows(M, run, min_rows=16)
+    return codes, scales
+
+
+def gemm_mxfp4_f64(a_codes, a_scales, b_codes, b_scales, rows=None) -> np.ndarray:
+    """Y[rows, N] = sum_k E2M1(a) 2^(sa-127) E2M1(b) 2^(sb-127) in FP64."""
+    a_codes, a_scales = np.ascontiguousarray(a_codes), np.ascontiguousarray(a_scales)
+    b_codes, b_scales = np.ascontiguousarray(b_codes), np.ascontiguousarray(b_scales)
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    N = b_codes.shape[0]
+    rows = _rows_arg(rows, M)
+    y = np.zeros((rows.size, N), np.float64)
+    L = lib()
+
+    def run(t0, t1):
+        L.oracle_gemm_mxfp4_f64(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), N, K,
+                                _ptr(rows[t0:t1]) if t1 > t0 else None, t1 - t0,
+                                y[t0:].ctypes.data_as(ctypes.c_void_p))
+
+    _split_rows(rows.size, run)
+    return y
 
 
 def dequant(codes, sf) -> np.ndarray:

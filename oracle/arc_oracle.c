@@ -527,6 +527,75 @@ void oracle_quantize_fp8_rows(const uint16_t* x, int64_t K, int64_t ldx, float s
     for (int64_t k = 0; k < K; ++k) codes[m * ldc + k] = oracle_e4m3_encode_signed(bf16_to_f32(x[m * ldx + k]) / s);
 }
 
+/* ------------------------------------------------------------------------------------------ */
+/* MXFP4 ("ARCQuant", Methodologie: the approach extends to the MXFP4 format), read as the OCP  */
+/* microscaling format: blocks of 32 consecutive values share one power-of-two scale X =        */
+/* 2^(floor(log2(amax_block)) - 2) (2 = the largest E2M1 exponent), stored as E8M0 = exponent + */
+/* 127 clamped to [0, 254]; elements are E2M1_rn_sat(x / X) with the sign kept on zero, as for  */
+/* NVFP4. An all-zero block has scale byte 0 and zero codes. No tensor scale.                  */
+/* ------------------------------------------------------------------------------------------ */
+
+uint8_t oracle_mxfp4_scale_byte(float amax) {
+  if (!(amax > 0.0f)) return 0;
+  int e2 = 0;
+  (void)frexpf(amax, &e2); /* amax = f * 2^e2, f in [0.5, 1): floor(log2(amax)) = e2 - 1 */
+  int e = (e2 - 1) - 2;
+  if (e < -127) e = -127;
+  if (e > 127) e = 127;
+  return (uint8_t)(e + 127);
+}
+
+void oracle_quantize_mxfp4_rows(const uint16_t* x, int64_t K, int64_t ldx, uint8_t* codes, uint8_t* scales,
+                                int64_t m0, int64_t m1) {
+  const int64_t nb = K / 32;
+  for (int64_t m = m0; m < m1; ++m) {
+    const uint16_t* row = x + m * ldx;
+    for (int64_t b = 0; b < nb; ++b) {
+      float v[32];
+      float amax = 0.0f;
+      for (int i = 0; i < 32; ++i) {
+        v[i] = bf16_to_f32(row[32 * b + i]);
+        if (fabsf(v[i]) > amax) amax = fabsf(v[i]);
+      }
+      const uint8_t sb = oracle_mxfp4_scale_byte(amax);
+      scales[m * nb + b] = sb;
+      for (int i = 0; i < 32; i += 2) {
+        uint8_t lo = 0, hi = 0;
+        if (amax > 0.0f) {
+          /* x / 2^(sb - 127): exact in fp32 for every bf16 x (a power-of-two scaling) */
+          lo = oracle_e2m1_encode(ldexpf(v[i], 127 - (int)sb));
+          hi = oracle_e2m1_encode(ldexpf(v[i + 1], 127 - (int)sb));
+        }
+        codes[m * (K / 2) + (32 * b + i) / 2] = (uint8_t)(lo | (hi << 4));
+      }
+    }
+  }
+}
+
+/* Y[rows[t], n] = sum_k E2M1(a) 2^(sa - 127) E2M1(b) 2^(sb - 127) in FP64 (exact per product). */
+void oracle_gemm_mxfp4_f64(const uint8_t* a_codes, const uint8_t* a_sc, const uint8_t* b_codes, const uint8_t* b_sc,
+                           int64_t N, int64_t K, const int64_t* rows, int64_t nrows, double* y) {
+  const int64_t nb = K / 32;
+  for (int64_t t = 0; t < nrows; ++t) {
+    const int64_t m = rows[t];
+    for (int64_t n = 0; n < N; ++n) {
+      double acc = 0.0;
+      for (int64_t b = 0; b < nb; ++b) {
+        const double sa = ldexp(1.0, (int)a_sc[m * nb + b] - 127), sw = ldexp(1.0, (int)b_sc[n * nb + b] - 127);
+        double part = 0.0;
+        for (int i = 0; i < 32; ++i) {
+          const int64_t k = 32 * b + i;
+          const uint8_t ca = (uint8_t)((a_codes[m * (K / 2) + k / 2] >> (4 * (k & 1))) & 15);
+          const uint8_t cb = (uint8_t)((b_codes[n * (K / 2) + k / 2] >> (4 * (k & 1))) & 15);
+          part += (double)oracle_e2m1_decode(ca) * (double)oracle_e2m1_decode(cb);
+        }
+        acc += part * sa * sw;
+      }
+      y[t * N + n] = acc;
+    }
+  }
+}
+
 void oracle_e4m3_decode_array(const uint8_t* c, int64_t n, float* out) {
   for (int64_t i = 0; i < n; ++i) out[i] = oracle_e4m3_decode(c[i]);
 }
