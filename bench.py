@@ -681,6 +681,7 @@ def main():
             ap.error("--reorder applies to the NVFP4 format")
         for L in layers:
             L["r"], L["fp8"] = 0, True
+        desc = f"{desc}; run in FP8 W8A8 (per-tensor scales, no residual channels)"
     if args.impl == "reference":
         if layers is None:
             if rank == 0:
