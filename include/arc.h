@@ -353,7 +353,13 @@ arc_status arc_debug_inject(int32_t kind);
  *          8 bytes per row: up to about 580 000 rows; larger requests return ARC_ERR_WORKSPACE
  *          before any launch.
  *   Set-up: the first call on a device looks up the array's device address on that device (it
- *          must be the current device); make that first call before any stream capture.
+ *          must be the current device) and keeps it for the life of the process; make that first
+ *          call before any stream capture. The kept address is not looked up again, so it is not
+ *          valid after cudaDeviceReset (or any other teardown of the device's primary context):
+ *          do not call this entry point on a device after resetting it.
+ *   Errors: argument, shape and alignment errors are reported first, in the same order as
+ *          arc_quantize_act_nvfp4 reports them; ARC_ERR_WORKSPACE (request beyond the array)
+ *          comes after them.
  *   Sharing: every call uses the same array and leaves its last contents in it; nothing in the
  *          array needs to start at zero. Calls whose work overlaps on the GPU (other streams,
  *          other host threads) race on the array and must be ordered by the caller.

@@ -147,7 +147,7 @@ __device__ __forceinline__ uint4 lds_u32x4(uint32_t addr) {
   return v;
 }
 
-constexpr int kGemmThreads = 480;  // producer, 2 MMA issuers, 4 scale writers, 8 epilogue warps
+constexpr int kGemmThreads = 480;  // producer, MMA issuer, idle warp, 4 scale writers, 8 epilogue warps
 constexpr int kGemmEpiWarp0 = 7;
 
 template <int KIND, bool ADD>

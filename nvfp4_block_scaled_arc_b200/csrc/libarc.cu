@@ -156,10 +156,11 @@ QuantWs carve_quant_ws(void* ws) {
 // Quantization driver shared by activations and weights, in the natural channel order (idx lists
 // the outlier channels) or reordered (perm != nullptr: primary channel p is input channel perm[p]
 // and the outlier channels are perm[0 .. r)).
-arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, const int32_t* idx, int32_t r,
-                           const void* gain, float eps, const float* static_scale, uint8_t* codes, uint8_t* sf,
-                           float* scale_out, void* workspace, size_t ws_bytes, arc_stream_t stream, int dup,
-                           const int32_t* perm = nullptr) {
+// The checks of the quantizer's arguments that need neither the workspace nor the device, in the
+// order every quantizer entry point reports them.
+arc_status quantize_check(const void* x, int64_t M, int64_t K, int64_t ldx, const int32_t* idx, int32_t r,
+                          const void* gain, uint8_t* codes, uint8_t* sf, float* scale_out,
+                          const int32_t* perm) {
   if (!x || !codes || !sf || !scale_out) return ARC_ERR_INVALID_ARG;
   if (M <= 0 || K <= 0 || K % 16 || r < 0 || r % 16 || r > K || ldx < K) return ARC_ERR_INVALID_ARG;
   if (!perm && r > 0 && !idx) return ARC_ERR_INVALID_ARG;
@@ -168,10 +169,20 @@ arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, con
   if (smem > static_cast<size_t>(perm ? arc::kQReoSmemMax : arc::kQRowsSmemMax)) return ARC_ERR_UNSUPPORTED;
   if (!al16(x) || (ldx * 2) % 16 || !al16(codes) || !al16(sf) || (gain && !al16(gain)) || (perm && !al16(perm)))
     return ARC_ERR_ALIGNMENT;
+  return ARC_OK;
+}
+
+arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, const int32_t* idx, int32_t r,
+                           const void* gain, float eps, const float* static_scale, uint8_t* codes, uint8_t* sf,
+                           float* scale_out, void* workspace, size_t ws_bytes, arc_stream_t stream, int dup,
+                           const int32_t* perm = nullptr) {
+  arc_status st = quantize_check(x, M, K, ldx, idx, r, gain, codes, sf, scale_out, perm);
+  if (st != ARC_OK) return st;
+  const size_t smem = perm ? arc::qreo_smem_bytes(static_cast<int>(K)) : arc::qrows_smem_bytes(static_cast<int>(K), r);
   if (!workspace || ws_bytes < arc_quantize_workspace_bytes(M, r)) return ARC_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ARC_ERR_ALIGNMENT;
   int sms = 0;
-  arc_status st = device_check(&sms);
+  st = device_check(&sms);
   if (st != ARC_OK) return st;
   cudaStream_t s = S(stream);
   QuantWs w = carve_quant_ws(workspace);
@@ -747,10 +758,12 @@ arc_status arc_quantize_act_nvfp4_static_scratch(const void* x_bf16, int64_t M, 
                                                  const int32_t* d_idx, int32_t r, const void* rms_gain_bf16,
                                                  float rms_eps, const float* d_static_scale, uint8_t* codes,
                                                  uint8_t* sf, float* d_scale_out, arc_stream_t stream) {
-  if (M <= 0 || r < 0) return ARC_ERR_INVALID_ARG;
+  // argument errors first, in the order of the workspace entry point, then the array's limit
+  arc_status st = quantize_check(x_bf16, M, K, ldx, d_idx, r, rms_gain_bf16, codes, sf, d_scale_out, nullptr);
+  if (st != ARC_OK) return st;
   if (arc_quantize_workspace_bytes(M, r) > static_cast<size_t>(ARC_STATIC_SCRATCH_BYTES)) return ARC_ERR_WORKSPACE;
   void* ws = nullptr;
-  const arc_status st = static_scratch_address(&ws);
+  st = static_scratch_address(&ws);
   if (st != ARC_OK) return st;
   return quantize_common(x_bf16, M, K, ldx, d_idx, r, rms_gain_bf16, rms_eps, d_static_scale, codes, sf,
                          d_scale_out, ws, ARC_STATIC_SCRATCH_BYTES, stream, 0);

@@ -97,3 +97,19 @@ def test_host_checks_of_the_reorder_fp8_and_schedule_calls(L):
     assert L.arc_gemm_fp8(fake, 64, fake, fake, 64, fake, 4, 12, 64, fake, 16, None, 0, None) == 1
     # schedule driver: T > 0 steps and no flags
     assert L.arc_recurrent_prefill_schedule(fake, 16, None, 4, None, ws, 1 << 20, None) == 1
+
+
+def test_static_scratch_reports_argument_errors_before_its_size_limit(L):
+    # a request that is both too large for the fixed array and malformed reports the argument
+    # error first, like the workspace entry point does
+    P = ctypes.c_void_p
+    fake = P(0x10000)
+    big = 1 << 22  # rows: far beyond the array's limit
+    assert L.arc_quantize_act_nvfp4_static_scratch(fake, big, 40, 40, None, 0, None, 1e-6, None, fake, fake, fake,
+                                                   None) == 1  # K % 16 != 0
+    assert L.arc_quantize_act_nvfp4_static_scratch(fake, big, 64, 64, None, 16, None, 1e-6, None, fake, fake, fake,
+                                                   None) == 1  # r > 0 without idx
+    assert L.arc_quantize_act_nvfp4_static_scratch(fake, big, 64, 64, None, 0, None, 1e-6, None, P(0x10008), fake,
+                                                   fake, None) == 2  # misaligned codes
+    assert L.arc_quantize_act_nvfp4_static_scratch(fake, big, 64, 64, None, 0, None, 1e-6, None, fake, fake, fake,
+                                                   None) == 6  # well-formed, too large

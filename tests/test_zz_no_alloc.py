@@ -6,7 +6,8 @@ to its host framework's allocator). It takes its temporary space from a fixed ar
 library instead of a workspace argument. This test calls both entry points through the C ABI on
 the same inputs, twice in a row with different inputs (the second call finds the first call's
 leftovers in the shared array), and requires identical codes, scale bytes and tensor scales.
-It also checks that a request larger than the array is refused before any launch.
+It also checks that a request larger than the array is refused before any launch, and that
+repeated calls leave the device's free memory unchanged (the call allocates nothing).
 """
 import ctypes
 
@@ -86,3 +87,33 @@ def test_static_scratch_refuses_requests_beyond_its_size():
         ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(scale.data_ptr()),
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == ARC_ERR_WORKSPACE
+
+
+def test_static_scratch_allocates_no_device_memory():
+    L = arc.lib()
+    d = W.llama8b("o", rows=512, with_w=False)
+    x = _dev(d["x"])
+    r = 128
+    idx = arc.calibrate_outliers(x, r)
+    M, K = x.shape
+    codes = torch.empty(arc.codes_bytes(M, K + r), dtype=torch.uint8, device="cuda")
+    sf = torch.empty(arc.sf_bytes(M, K + r), dtype=torch.uint8, device="cuda")
+    scale = torch.zeros(1, dtype=torch.float32, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+    def call():
+        st = L.arc_quantize_act_nvfp4_static_scratch(
+            ctypes.c_void_p(x.data_ptr()), M, K, K, ctypes.c_void_p(idx.data_ptr()), r, None, 1e-6, None,
+            ctypes.c_void_p(codes.data_ptr()), ctypes.c_void_p(sf.data_ptr()), ctypes.c_void_p(scale.data_ptr()),
+            stream)
+        assert st == 0, st
+
+    call()  # the first call looks up the array's address
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(5):
+        call()
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, (free0, free1)
+    assert arc.last_device_status() == 0
