@@ -76,6 +76,7 @@ def lib():
                 "oracle_sf_swizzle": (None, [P, I64, I64, P]),
                 "oracle_sf_unswizzle": (None, [P, I64, I64, P]),
                 "oracle_gemm_nvfp4_f64": (None, [P, P, F, P, P, F, I64, I64, P, I64, I64, I64, P]),
+                "oracle_quantize_mxfp4_arc_rows": (None, [P, I64, I64, P, I32, I32, P, P, P, I64, I64]),
                 "oracle_gemm_nvfp4_i64": (None, [P, P, P, P, I64, I64, P, I64, I64, I64, P]),
                 "oracle_gemm_bf16_f64": (None, [P, I64, P, I64, I64, I64, P, I64, P]),
                 "oracle_channel_absmax": (None, [P, I64, I64, I64, P]),
@@ -366,6 +367,40 @@ def quantize_mxfp4(x):
 
     _split_rows(M, run, min_rows=16)
     return codes, scales
+
+
+def _mxfp4_arc(x, idx, dup: bool, want_residual: bool = False):
+    x = as_u16(x)
+    M, K = x.shape
+    idx = np.ascontiguousarray(np.asarray(idx, dtype=np.int32).reshape(-1))
+    r = idx.size
+    assert K % 32 == 0 and r % 32 == 0 and r <= K
+    kp = kpad(K + r)
+    codes = np.zeros((M, kp // 2), np.uint8)
+    scales = np.zeros((M, kp // 32), np.uint8)
+    res = np.zeros((M, r), np.float32) if (want_residual and r > 0) else None
+    L = lib()
+
+    def run(r0, r1):
+        L.oracle_quantize_mxfp4_arc_rows(_ptr(x), K, K, _ptr(idx) if r else None, r, 1 if dup else 0, _ptr(codes),
+                                         _ptr(scales), _ptr(res) if res is not None else None, r0, r1)
+
+    _split_rows(M, run, min_rows=16)
+    if want_residual:
+        return codes, scales, (res if res is not None else np.zeros((M, 0), np.float32))
+    return codes, scales
+
+
+def quantize_act_mxfp4(x, idx, want_residual: bool = False):
+    """MXFP4 with augmented residual channels (arc_oracle.c, MXFP4 with augmented residual
+    channels): X [M, K] bf16 -> (codes [M, K_pad/2], canonical E8M0 scale bytes [M, K_pad/32]
+    [, residuals [M, r] f32]); K and r multiples of 32."""
+    return _mxfp4_arc(x, idx, dup=False, want_residual=want_residual)
+
+
+def pack_weight_mxfp4(w, idx):
+    """W_aug = [W | W[:, idx]] in MXFP4: (codes [N, K_pad/2], canonical scale bytes [N, K_pad/32])."""
+    return _mxfp4_arc(w, idx, dup=True)
 
 
 def gemm_mxfp4_f64(a_codes, a_scales, b_codes, b_scales, rows=None) -> np.ndarray:

@@ -572,6 +572,61 @@ void oracle_quantize_mxfp4_rows(const uint16_t* x, int64_t K, int64_t ldx, uint8
   }
 }
 
+/* ------------------------------------------------------------------------------------------ */
+/* MXFP4 with augmented residual channels ("ARCQuant", Resultaten / Generaliseerbaarheid: the   */
+/* approach extends to MXFP4): the dual-stage code with MXFP4 blocks in place of NVFP4 blocks.  */
+/*   primary   MXFP4 of the row in blocks of 32 consecutive channels (the code above);          */
+/*   residual  for outlier channel c = idx[j]: x_c - E2M1(code_c) * X_b(c), fp32 multiply (exact: */
+/*             X is a power of two) then fp32 subtract; the residuals in idx order form r/32    */
+/*             blocks coded the same way and written at columns K + j;                          */
+/*   weights   append the duplicated channels W[:, idx] instead (re-blocked among themselves).  */
+/* K % 32 == 0, r % 32 == 0; K_pad = K + r rounded up to 64 (one tensor-core K step); padding   */
+/* codes and scale bytes are 0. Scale bytes canonical: [rows, K_pad / 32].                      */
+/* ------------------------------------------------------------------------------------------ */
+
+/* One 32-value block: its scale byte, its codes and its scale X = 2^(byte - 127). */
+static void mxfp4_block(const float* v, uint8_t* c32, uint8_t* sb_out, float* X_out) {
+  float amax = 0.0f;
+  for (int i = 0; i < 32; ++i)
+    if (fabsf(v[i]) > amax) amax = fabsf(v[i]);
+  const uint8_t sb = oracle_mxfp4_scale_byte(amax);
+  for (int i = 0; i < 32; ++i) c32[i] = amax > 0.0f ? oracle_e2m1_encode(ldexpf(v[i], 127 - (int)sb)) : 0;
+  *sb_out = sb;
+  if (X_out) *X_out = ldexpf(1.0f, (int)sb - 127);
+}
+
+void oracle_quantize_mxfp4_arc_rows(const uint16_t* x, int64_t K, int64_t ldx, const int32_t* idx, int32_t r,
+                                    int32_t dup_mode, uint8_t* codes, uint8_t* sc, float* res_out, int64_t m0,
+                                    int64_t m1) {
+  const int64_t kpad = kpad_of(K + r);
+  float* row = (float*)malloc(sizeof(float) * (size_t)K);
+  float* X_blk = (float*)malloc(sizeof(float) * (size_t)(K / 32 + 1));
+  float ext[32];
+  uint8_t c32[32];
+  for (int64_t m = m0; m < m1; ++m) {
+    for (int64_t k = 0; k < K; ++k) row[k] = bf16_to_f32(x[m * ldx + k]);
+    uint8_t* crow = codes + m * (kpad / 2);
+    uint8_t* srow = sc + m * (kpad / 32);
+    memset(crow, 0, (size_t)(kpad / 2));
+    memset(srow, 0, (size_t)(kpad / 32));
+    for (int64_t b = 0; b < K / 32; ++b) {
+      mxfp4_block(row + 32 * b, c32, &srow[b], &X_blk[b]);
+      for (int i = 0; i < 32; ++i) put_code(crow, 32 * b + i, c32[i]);
+    }
+    for (int32_t jb = 0; jb < r / 32; ++jb) {
+      for (int i = 0; i < 32; ++i) {
+        const int32_t c = idx[32 * jb + i];
+        ext[i] = dup_mode ? row[c] : row[c] - oracle_e2m1_decode(oracle_get_code(crow, c)) * X_blk[c / 32];
+        if (res_out) res_out[m * r + 32 * jb + i] = ext[i];
+      }
+      mxfp4_block(ext, c32, &srow[K / 32 + jb], NULL);
+      for (int i = 0; i < 32; ++i) put_code(crow, K + 32 * jb + i, c32[i]);
+    }
+  }
+  free(row);
+  free(X_blk);
+}
+
 /* Y[rows[t], n] = sum_k E2M1(a) 2^(sa - 127) E2M1(b) 2^(sb - 127) in FP64 (exact per product). */
 void oracle_gemm_mxfp4_f64(const uint8_t* a_codes, const uint8_t* a_sc, const uint8_t* b_codes, const uint8_t* b_sc,
                            int64_t N, int64_t K, const int64_t* rows, int64_t nrows, double* y) {

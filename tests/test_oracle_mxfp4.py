@@ -88,3 +88,150 @@ def test_gemm_equals_textbook_matmul_on_representable_inputs():
     bc, bsc = O.quantize_mxfp4(_bits(xw))
     y = O.gemm_mxfp4_f64(ac, asc, bc, bsc)
     np.testing.assert_allclose(y, xa.astype(np.float64) @ xw.astype(np.float64).T, rtol=1e-14, atol=0)
+
+
+# ---------------------------------------------------------------------------------------------
+# MXFP4 with augmented residual channels (ARCQuant, Resultaten / Generaliseerbaarheid: the
+# approach extends to MXFP4): the dual-stage code with 32-value MXFP4 blocks. Each pin below is
+# built without the C code's block routine, so a slip in it (a wrong block, a dropped residual
+# term, the wrong scale of the deducted value) fails one of them.
+# ---------------------------------------------------------------------------------------------
+
+MIDS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+
+
+def _np_e2m1(v):
+    """Independent E2M1 encoder: nearest grid magnitude, ties to the even code, saturation at
+    6, sign bit from the sign of v (also for values that round to zero)."""
+    v = np.asarray(v, np.float64)
+    m = np.abs(v)
+    code = np.searchsorted(MIDS, m, side="left")  # number of midpoints strictly below m
+    tie = np.isin(m, MIDS)
+    code = np.where(tie & (code % 2 == 1), code + 1, code)  # on a midpoint, take the even neighbour
+    code = np.minimum(code, 7)
+    return (code | np.where(np.signbit(v), 8, 0)).astype(np.uint8)
+
+
+def _np_mxfp4_blocks(vals):
+    """Independent MXFP4 of fp32 rows (K % 32 == 0): codes [M, K] (one per element) and scale
+    bytes [M, K/32], the scale exponent from frexp."""
+    v = np.asarray(vals, np.float32)
+    M, K = v.shape
+    blk = v.reshape(M, K // 32, 32)
+    amax = np.abs(blk).max(axis=2).astype(np.float64)
+    _, e2 = np.frexp(amax)
+    sb = np.where(amax > 0, np.clip(e2 - 1 - 2 + 127, 0, 254), 0).astype(np.int64)
+    scaled = np.ldexp(blk, (127 - sb)[:, :, None].astype(np.int32)).astype(np.float32)
+    codes = np.where((amax > 0)[:, :, None], _np_e2m1(scaled), 0).astype(np.uint8)
+    return codes.reshape(M, K), sb.astype(np.uint8)
+
+
+def _unpack(codes):
+    lo, hi = codes & 15, codes >> 4
+    return np.stack([lo, hi], axis=2).reshape(codes.shape[0], -1)
+
+
+def _deq(c, sb):
+    X = np.ldexp(1.0, np.repeat(sb.astype(np.int64) - 127, 32, axis=1))
+    return np.where(c & 8, -1.0, 1.0) * E2M1[c & 7] * X
+
+
+def test_np_encoder_agrees_with_the_plain_oracle_block():
+    rng = np.random.default_rng(10)
+    v = (rng.standard_t(3, size=(20, 256)) * np.exp(rng.uniform(-8, 8, size=(20, 1)))).astype(np.float32)
+    x = _bits(v)
+    codes, sc = O.quantize_mxfp4(x)
+    c_np, sb_np = _np_mxfp4_blocks(O.bf16_bits_to_f32(x))
+    np.testing.assert_array_equal(sc, sb_np)
+    np.testing.assert_array_equal(_unpack(codes), c_np)
+
+
+def test_arc_without_channels_is_plain_mxfp4():
+    rng = np.random.default_rng(11)
+    x = _bits(rng.standard_normal((33, 512)))
+    c0, s0 = O.quantize_mxfp4(x)
+    c1, s1 = O.quantize_act_mxfp4(x, np.zeros(0, np.int32))
+    np.testing.assert_array_equal(c0, c1)
+    np.testing.assert_array_equal(s0, s1)
+
+
+def test_weight_pack_equals_mxfp4_of_the_explicit_augmented_matrix():
+    rng = np.random.default_rng(12)
+    N, K, r = 24, 320, 64  # K + r = 384: no padding; also check a padded case below
+    for K, r in ((320, 64), (256, 32)):
+        w = _bits(rng.standard_normal((N, K)) * 0.02)
+        idx = rng.choice(K, size=r, replace=False).astype(np.int32)
+        kp = (K + r + 63) // 64 * 64
+        waug = np.zeros((N, kp), np.uint16)
+        waug[:, :K] = w
+        waug[:, K:K + r] = w[:, idx]
+        c_ref, s_ref = O.quantize_mxfp4(waug)
+        c, s = O.pack_weight_mxfp4(w, idx)
+        np.testing.assert_array_equal(c, c_ref)
+        np.testing.assert_array_equal(s, s_ref)
+
+
+def test_activation_residual_blocks_against_an_independent_construction():
+    rng = np.random.default_rng(13)
+    M, K, r = 40, 512, 64
+    v = rng.standard_normal((M, K)).astype(np.float32)
+    hot = rng.choice(K, size=12, replace=False)
+    v[:, hot] *= rng.uniform(20, 80, size=12).astype(np.float32)
+    x = _bits(v)
+    xf = O.bf16_bits_to_f32(x)
+    idx = np.argsort(-np.abs(xf).max(axis=0), kind="stable")[:r].astype(np.int32)
+    codes, sc, res = O.quantize_act_mxfp4(x, idx, want_residual=True)
+    # primary part: plain MXFP4 of X
+    cp, sp = O.quantize_mxfp4(x)
+    np.testing.assert_array_equal(codes[:, :K // 2], cp)
+    np.testing.assert_array_equal(sc[:, :K // 32], sp)
+    # residual of each outlier channel: x - E2M1(code) * X in fp32 (the product is exact)
+    deq = _deq(_unpack(cp), sp).astype(np.float32)
+    R = (xf[:, idx] - deq[:, idx]).astype(np.float32)
+    np.testing.assert_array_equal(res, R)
+    c_np, sb_np = _np_mxfp4_blocks(R)
+    np.testing.assert_array_equal(_unpack(codes)[:, K:K + r], c_np)
+    np.testing.assert_array_equal(sc[:, K // 32:(K + r) // 32], sb_np)
+    # padding to K_pad is zero
+    assert not _unpack(codes)[:, K + r:].any() and not sc[:, (K + r) // 32:].any()
+
+
+def test_residual_never_increases_the_error_and_vanishes_on_representable_rows():
+    rng = np.random.default_rng(14)
+    M, K, r = 30, 256, 32
+    x = _bits(rng.standard_t(3, size=(M, K)) * 3)
+    xf = O.bf16_bits_to_f32(x).astype(np.float64)
+    idx = rng.choice(K, size=r, replace=False).astype(np.int32)
+    codes, sc = O.quantize_act_mxfp4(x, idx)
+    c = _unpack(codes)
+    deq_main = _deq(c[:, :K], sc[:, :K // 32])[:, idx]
+    deq_res = _deq(c[:, K:K + r], sc[:, K // 32:(K + r) // 32])
+    e_plain = np.abs(xf[:, idx] - deq_main)
+    e_arc = np.abs(xf[:, idx] - deq_main - deq_res)
+    assert np.all(e_arc <= e_plain)
+    assert e_arc.sum() < e_plain.sum()
+    # representable rows leave zero residuals: appended codes and scale bytes all zero
+    mags = E2M1[rng.integers(0, 8, size=(M, K))]
+    mags[:, ::32] = 6.0
+    rep = (mags * np.ldexp(1.0, np.repeat(rng.integers(-5, 5, size=(M, K // 32)), 32, axis=1))).astype(np.float32)
+    c2, s2 = O.quantize_act_mxfp4(_bits(rep), idx)
+    assert not c2[:, K // 2:].any() and not s2[:, K // 32:].any()
+
+
+def test_augmented_gemm_is_main_plus_correction():
+    rng = np.random.default_rng(15)
+    M, N, K, r = 12, 10, 256, 64
+    x = _bits(rng.standard_normal((M, K)))
+    w = _bits(rng.standard_normal((N, K)) * 0.02)
+    idx = rng.choice(K, size=r, replace=False).astype(np.int32)
+    ac, asc = O.quantize_act_mxfp4(x, idx)
+    bc, bsc = O.pack_weight_mxfp4(w, idx)
+    y = O.gemm_mxfp4_f64(ac, asc, bc, bsc)
+    a = _deq(_unpack(ac), asc)
+    b = _deq(_unpack(bc), bsc)
+    main = a[:, :K] @ b[:, :K].T
+    corr = a[:, K:K + r] @ b[:, K:K + r].T
+    np.testing.assert_allclose(y, main + corr, rtol=1e-12, atol=1e-30)
+    # the correction pairs each residual with its duplicated weight column
+    np.testing.assert_allclose(corr, a[:, K:K + r] @ _deq(_unpack(O.quantize_mxfp4(w[:, idx])[0]),
+                                                         O.quantize_mxfp4(w[:, idx])[1]).T, rtol=1e-12)
