@@ -29,7 +29,8 @@ Variants of the linear-layer workloads:
 Metric: NVFP4 ARC GEMM TFLOP/s = sum over the step of 2*M*N*(K+r) / step time, with the fused
 activation quantizer's GB/s (read X + write codes + scale bytes) beside it.
 Timing: CUDA events on the launching stream around every step and every kernel call; the L2 is
-flushed (a 256 MiB write) before every timed step, outside the events. Multi-GPU: one process
+flushed before every timed step, outside the events (a 256 MiB buffer written, then read back, so
+the lines it leaves in L2 are clean). Multi-GPU: one process
 per GPU, each rank runs the same step on its own token batch (weak scaling, no data-path
 collective); time = max over ranks.
 
@@ -54,6 +55,7 @@ import torch  # noqa: E402
 
 METRIC = "NVFP4 ARC GEMM TFLOP/s (% FP4 peak) + fused act-quant GB/s, 1×B200"
 METRIC_FP8 = "FP8 W8A8 GEMM TFLOP/s (% FP8 peak) + act-quant GB/s, 1×B200"
+METRIC_MX = "MXFP4 ARC GEMM TFLOP/s (% FP4 peak) + fused act-quant GB/s, 1×B200"
 UNIT = "TFLOP/s"
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLOP/s)
 
@@ -114,6 +116,8 @@ def layer_quant_bytes(L):
     if L.get("fp8"):
         return 3 * L["M"] * L["K"]
     kp = kpad(L["K"] + L["r"])
+    if L.get("mx"):  # one E8M0 byte per 32 values
+        return 2 * L["M"] * L["K"] + L["M"] * kp // 2 + L["M"] * kp // 32
     return 2 * L["M"] * L["K"] + L["M"] * kp // 2 + L["M"] * kp // 16
 
 
@@ -214,6 +218,13 @@ def _ev():
     return torch.cuda.Event(enable_timing=True)
 
 
+def flush_l2(buf):
+    """Write a buffer about twice the L2's size, then read it back: no input stays in L2, and the
+    lines left there are clean, so no write-back of the flush buffer lands in the timed work."""
+    buf.zero_()
+    buf.view(torch.int64).max()
+
+
 def _barrier(world):
     if world > 1:
         torch.distributed.barrier()
@@ -241,6 +252,8 @@ def run_layers(args, rank, world, device, layers, with_error=False):
     stream = torch.cuda.Stream(device=device)
     reorder = getattr(args, "reorder", False)
     fp8 = getattr(args, "format", "nvfp4") == "fp8"
+    mx = getattr(args, "format", "nvfp4") == "mxfp4"
+    gemm = arc.gemm_fp8 if fp8 else arc.gemm_mxfp4 if mx else arc.gemm_nvfp4
     xs_host, xs, idx, packed, qa, ys, wsp, errs = {}, {}, {}, {}, {}, {}, {}, {}
     rs = {L["name"]: L["r"] for L in layers}
 
@@ -249,6 +262,9 @@ def run_layers(args, rank, world, device, layers, with_error=False):
         # or NVFP4 reordered
         if fp8:
             return arc.quantize_fp8(xs[name], stream=stream, **kw)
+        if mx:
+            kw.pop("workspace", None)  # the MXFP4 quantizer needs none
+            return arc.quantize_act_mxfp4(xs[name], idx[name], stream=stream, **kw)
         if reorder:
             return arc.quantize_act_nvfp4_reordered(xs[name], idx[name], rs[name], stream=stream, **kw)
         return arc.quantize_act_nvfp4(xs[name], idx[name], stream=stream, **kw)
@@ -263,6 +279,9 @@ def run_layers(args, rank, world, device, layers, with_error=False):
             if fp8:
                 idx[name] = None
                 packed[name] = arc.quantize_fp8(w, stream=stream)  # weights: their own tensor scale
+            elif mx:
+                idx[name] = arc.calibrate_outliers(xs[name], r, stream=stream) if r else None
+                packed[name] = arc.pack_weight_mxfp4(w, idx[name], stream=stream)
             elif reorder:
                 # idx holds the full calibration order; its first r channels are the outliers
                 idx[name] = arc.calibrate_order(xs[name], stream=stream)
@@ -275,7 +294,7 @@ def run_layers(args, rank, world, device, layers, with_error=False):
             wsp[name] = torch.empty(arc.quantize_workspace_bytes(M, r), dtype=torch.uint8, device=device)
             if with_error:
                 # relative error of the NVFP4 + ARC output against the BF16 product of the inputs
-                y = (arc.gemm_fp8 if fp8 else arc.gemm_nvfp4)(qa[name], packed[name], stream=stream).float()
+                y = gemm(qa[name], packed[name], stream=stream).float()
                 yb = arc.gemm_bf16(xs[name], w, stream=stream).float()
                 errs[name] = (torch.linalg.norm(y - yb) / torch.linalg.norm(yb)).item()
             del w
@@ -291,14 +310,14 @@ def run_layers(args, rank, world, device, layers, with_error=False):
             quant(name, out=qa[name], workspace=wsp[name])
             if e1 is not None:
                 e1.record(stream)
-            (arc.gemm_fp8 if fp8 else arc.gemm_nvfp4)(qa[name], packed[name], out=ys[name], stream=stream)
+            gemm(qa[name], packed[name], out=ys[name], stream=stream)
             if e2 is not None:
                 e2.record(stream)
                 rec.append((e0, e1, e2))
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            flush.zero_()
+            flush_l2(flush)
             step(None)
     stream.synchronize()
     if arc.last_device_status(stream) != 0:
@@ -310,7 +329,7 @@ def run_layers(args, rank, world, device, layers, with_error=False):
     with ClockSampler(device) as clk:
         with torch.cuda.stream(stream):
             for _ in range(args.steps):
-                flush.zero_()
+                flush_l2(flush)
                 s0, s1 = _ev(), _ev()
                 s0.record(stream)
                 rec = []
@@ -348,7 +367,7 @@ def run_layers(args, rank, world, device, layers, with_error=False):
                 name = L["name"]
                 xs[name].copy_(xs_pin[name], non_blocking=True)
                 quant(name, out=qa[name], workspace=wsp[name])
-                (arc.gemm_fp8 if fp8 else arc.gemm_nvfp4)(qa[name], packed[name], out=ys[name], stream=stream)
+                gemm(qa[name], packed[name], out=ys[name], stream=stream)
                 ys_pin[name].copy_(ys[name], non_blocking=True)
 
         with torch.cuda.stream(stream):
@@ -380,16 +399,19 @@ def layers_line(args, world, layers, desc, res):
     value = step_flops * world * args.steps / (res["total_ms"] * 1e-3) / 1e12
     achieved = step_flops * args.steps / (res["g_ms"] * 1e-3) / 1e12
     quant_gbs = qbytes * args.steps / (res["q_ms"] * 1e-3) / 1e9
-    fp8 = getattr(args, "format", "nvfp4") == "fp8"
+    fmt = getattr(args, "format", "nvfp4")
+    fp8, mx = fmt == "fp8", fmt == "mxfp4"
     ratio = 2.0 if fp8 else FP4_OVER_BF16  # nominal dense FP8 / BF16 = 2, FP4 / BF16 = 4
     peak = pk["bf16_tflops"] * ratio
+    qkern = ("k_amax + k_quant_fp8" if fp8 else "k_quant_mx_rows" if mx else
+             "k_amax + k_quant_reordered" if getattr(args, "reorder", False) else "k_amax + k_quant_rows")
     return {
-        "metric": METRIC_FP8 if fp8 else METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC_FP8 if fp8 else METRIC_MX if mx else METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": res["total_ms"] / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3 x e4m3 -> f32 (bf16 out)" if fp8 else "e2m1 x e2m1 -> f32 (bf16 out)",
         "data": "synthetic (seeded; random weights and activations of the stated shapes)",
-        "config": {"workload": desc, "l2": "flushed (256 MiB write) before every step",
+        "config": {"workload": desc, "l2": "flushed before every step (256 MiB written, then read back)",
                    "parallelism": f"replicas x{world}",
                    "channel_order": "reordered by calibration abs-max" if getattr(args, "reorder", False)
                    else "natural (outlier list)"},
@@ -398,15 +420,14 @@ def layers_line(args, world, layers, desc, res):
         ("pct_fp8_peak" if fp8 else "pct_fp4_peak"): 100.0 * value / peak,
         "per_projection": res["per_layer"],
         "roofline": {"bound": "tensor",
-                     "kernel": f"k_gemm<{'fp8' if fp8 else 'nvfp4'}> (all {len(layers)} launches of a step)",
+                     "kernel": f"k_gemm<{fmt}> (all {len(layers)} launches of a step)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{src} bf16 burst {pk['bf16_tflops']} TFLOP/s x {ratio:g} "
                                     f"(nominal {'FP8' if fp8 else 'FP4'}/BF16 dense ratio)",
                      "traffic": ncu_traffic() if args.workload == "llama8b" and not getattr(args, "reorder", False)
-                     and not fp8 else None},
+                     and fmt == "nvfp4" else None},
         "quant_roofline": {"bound": "hbm",
-                           "kernel": "k_amax + " + ("k_quant_fp8" if fp8 else "k_quant_reordered"
-                                                    if getattr(args, "reorder", False) else "k_quant_rows"),
+                           "kernel": qkern,
                            "achieved": quant_gbs,
                            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": quant_gbs / pk["hbm_gbs"],
                            "peak_source": f"{src} copy bandwidth"},
@@ -469,7 +490,7 @@ def run_recurrent(args, rank, world, device):
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             for k in k_lows:
-                flush.zero_()
+                flush_l2(flush)
                 prefill(k)
     stream.synchronize()
     times = {k: [] for k in k_lows}
@@ -480,7 +501,7 @@ def run_recurrent(args, rank, world, device):
         with torch.cuda.stream(stream):
             for _ in range(args.steps):
                 for k in k_lows:
-                    flush.zero_()
+                    flush_l2(flush)
                     a, b = _ev(), _ev()
                     a.record(stream)
                     prefill(k)
@@ -501,6 +522,7 @@ def run_recurrent(args, rank, world, device):
                              "hidden_state_rel_err_vs_all_bf16": fidelity[k]}
     kk = 12 if 12 in ms else k_lows[-1]
     study = schedule_study(arc, h, h0, blk, wsp, flush, stream, T, kk, out[0], device)
+    contractive = contractive_study(arc, device, stream, T=T, budget=kk, r=r)
     # kernels per prefill: NVFP4 step = 2 x (2 quantizer launches + GEMM + SiLU + 2 quantizer
     # launches + GEMM), BF16 step = 2 x (RMSNorm + GEMM + SiLU + GEMM)
     launches = args.steps * sum(k * 2 * 7 + (T - k) * 2 * 4 for k in k_lows)
@@ -512,9 +534,82 @@ def run_recurrent(args, rank, world, device):
         "data": "synthetic (seeded; random weights and hidden state of the stated shapes)",
         "config": {"workload": f"recurrent SwiGLU block: S={S}, d={d}, ffn={F}, 2 pre-norm sublayers, T={T}, "
                                f"k_low in {k_lows}, r={r}",
-                   "l2": "flushed (256 MiB write) before every prefill", "parallelism": f"replicas x{world}"},
-        "per_k_low": per, "schedule_study": study, "clocks": clk.summary(), "e2e": None, "gpu_launches": launches,
+                   "l2": "flushed before every prefill (256 MiB written, then read back)", "parallelism": f"replicas x{world}"},
+        "per_k_low": per, "schedule_study": study, "contractive_study": contractive, "clocks": clk.summary(),
+        "e2e": None, "gpu_launches": launches,
     }
+
+
+def contractive_study(arc, device, stream, S=1024, d=2048, F=8192, T=16, budget=12, r=64, beta=0.5, eps=1.0,
+                      n_random=24):
+    """RAMP's placement result (section 3, Theorem 3.2: with locally contractive steps, low
+    precision early and BF16 late minimises the final-error bound; late placement maximises it;
+    random schedules fall between) checked on a block built to contract: the damped residual
+    h <- beta h + F(h) with beta = 1/2 and RMSNorm eps = 1 (n is then close to linear in h), the
+    recurrent workload's weights. The contraction factor is measured (BF16 step map, the ratio of
+    output to input perturbation norms); each schedule's final hidden-state error is against the
+    all-BF16 run. Fidelity only: nothing here is timed."""
+    import workloads as W
+
+    rec = W.recurrent(S=S, d=d, ffn=F)
+    with torch.cuda.stream(stream):
+        h0 = W.to_torch_bf16(rec["h"]).to(device)
+        subs = []
+        for L in rec["layers"]:
+            wgu, wd, gain = (W.to_torch_bf16(L[k]).to(device) for k in ("wgu", "wd", "gain"))
+            n = arc.rmsnorm_bf16(h0, gain, eps, stream=stream)
+            idx_gu = arc.calibrate_outliers(n, r, stream=stream)
+            act = arc.silu_mul_bf16(arc.gemm_bf16(n, wgu, stream=stream), stream=stream)
+            idx_d = arc.calibrate_outliers(act, r, stream=stream)
+            subs.append(dict(gain=gain, wgu=wgu, wd=wd, idx_gu=idx_gu, idx_d=idx_d,
+                             gu_q=arc.pack_weight_nvfp4(wgu, idx_gu, stream=stream),
+                             d_q=arc.pack_weight_nvfp4(wd, idx_d, stream=stream)))
+        blk = arc.RecurrentBlock(d, F, eps, subs, beta)
+        ws = torch.empty(blk.workspace_bytes(S), dtype=torch.uint8, device=device)
+
+        def run(flags, h_in=None):
+            h = (h0 if h_in is None else h_in).clone()
+            arc.recurrent_prefill_schedule(h, blk, flags, workspace=ws, stream=stream)
+            return h
+
+        # contraction factor of the BF16 step map along the reference trajectory
+        rng = torch.Generator(device="cpu").manual_seed(7)
+        rho, h = [], h0.clone()
+        for t in range(T):
+            dlt = (torch.randn(h.shape, generator=rng) * 1e-2 * h.float().pow(2).mean().sqrt().item()).to(device)
+            hp = (h.float() + dlt).bfloat16()
+            a, b = run([0], h), run([0], hp)
+            rho.append((torch.linalg.norm(b.float() - a.float()) / torch.linalg.norm(hp.float() - h.float())).item())
+            h = a
+        ref = run([0] * T).float()
+
+        def err(flags):
+            return (torch.linalg.norm(run(flags).float() - ref) / torch.linalg.norm(ref)).item()
+
+        k = T - budget
+        sch = {"ramp": [1] * budget + [0] * k, "early_bf16": [0] * k + [1] * budget,
+               "interleaved": [0 if (t % (T // k)) == T // k - 1 else 1 for t in range(T)]}
+        gen = np.random.default_rng(11)
+        seen = {tuple(v) for v in sch.values()}
+        rand = []
+        while len(rand) < n_random:
+            f = np.zeros(T, np.int64)
+            f[gen.choice(T, size=budget, replace=False)] = 1
+            if tuple(f.tolist()) not in seen:
+                seen.add(tuple(f.tolist()))
+                rand.append(f.tolist())
+        out = {name: {"schedule": "".join("L" if f else "B" for f in flags), "err": err(flags)}
+               for name, flags in sch.items()}
+        rerr = [err(f) for f in rand]
+    stream.synchronize()
+    if arc.last_device_status(stream) != 0:
+        raise RuntimeError("device status set during the contractive study")
+    return {"block": f"damped residual beta={beta}, RMSNorm eps={eps}, S={S}, d={d}, ffn={F}, r={r}, T={T}, "
+                     f"{budget} NVFP4 + {k} BF16 steps",
+            "contraction_factor": {"median": statistics.median(rho), "max": max(rho)},
+            "schedules": out,
+            "random": {"n": n_random, "min": min(rerr), "median": statistics.median(rerr), "max": max(rerr)},
+            "ordering_holds": out["ramp"]["err"] <= min(rerr) and max(rerr) <= out["early_bf16"]["err"]}
 
 
 def schedule_study(arc, h, h0, blk, wsp, flush, stream, T, budget, ref, device, reps=5):
@@ -538,7 +633,7 @@ def schedule_study(arc, h, h0, blk, wsp, flush, stream, T, budget, ref, device, 
             err = (torch.linalg.norm(h.float() - ref) / torch.linalg.norm(ref)).item()
             ts = []
             for _ in range(reps):
-                flush.zero_()
+                flush_l2(flush)
                 h.copy_(h0)
                 a, b = _ev(), _ev()
                 a.record(stream)
@@ -558,16 +653,21 @@ def schedule_study(arc, h, h0, blk, wsp, flush, stream, T, budget, ref, device, 
 # Oracle arm (CPU)
 # ---------------------------------------------------------------------------------------------
 
-def oracle_cache(layers, n_rows: int, reorder: bool = False, fp8: bool = False):
+def oracle_cache(layers, n_rows: int, reorder: bool = False, fmt: str = "nvfp4"):
     import oracle as O
 
     cache = {}
     for L in layers:
         d = L["gen"](n_rows, 0)
         x = d["x"][:n_rows]
-        if fp8:
+        if fmt == "mxfp4":
+            idx = O.calibrate(x, L["r"]) if L["r"] else np.zeros(0, np.int32)
+            bc, bsc = O.pack_weight_mxfp4(d["w"], idx)
+            cache[L["name"]] = dict(x=x, idx=idx, bc=bc, bsc=bsc, fmt=fmt)
+            continue
+        if fmt == "fp8":
             sa, sw = O.fp8_scale(O.amax(x)), O.fp8_scale(O.amax(d["w"]))
-            cache[L["name"]] = dict(x=x, sa=sa, sw=sw, bc=O.quantize_fp8(d["w"], sw), fp8=True)
+            cache[L["name"]] = dict(x=x, sa=sa, sw=sw, bc=O.quantize_fp8(d["w"], sw), fmt=fmt)
             continue
         sa = O.tensor_scale(O.amax(x))
         sw = O.tensor_scale(O.amax(d["w"]))
@@ -577,7 +677,7 @@ def oracle_cache(layers, n_rows: int, reorder: bool = False, fp8: bool = False):
         else:
             idx = O.calibrate(x, L["r"]) if L["r"] else np.zeros(0, np.int32)
             bc, bsf = O.pack_weight(d["w"], idx, sw)  # every output column needs the full weight
-        cache[L["name"]] = dict(x=x, idx=idx, sa=sa, sw=sw, bc=bc, bsf=bsf, reorder=reorder, fp8=False)
+        cache[L["name"]] = dict(x=x, idx=idx, sa=sa, sw=sw, bc=bc, bsf=bsf, reorder=reorder, fmt=fmt)
     return cache
 
 
@@ -590,7 +690,12 @@ def oracle_sample_step(layers, rows: int, cache: dict):
     flops = 0.0
     for L in layers:
         c = cache[L["name"]]
-        if c["fp8"]:
+        if c["fmt"] == "mxfp4":
+            ac, asc = O.quantize_act_mxfp4(c["x"][:rows], c["idx"])
+            O.gemm_mxfp4_f64(ac, asc, c["bc"], c["bsc"])
+            flops += 2.0 * rows * L["N"] * (L["K"] + L["r"])
+            continue
+        if c["fmt"] == "fp8":
             O.gemm_fp8_f64(O.quantize_fp8(c["x"][:rows], c["sa"]), c["sa"], c["bc"], c["sw"])
             flops += 2.0 * rows * L["N"] * L["K"]
             continue
@@ -603,13 +708,13 @@ def oracle_sample_step(layers, rows: int, cache: dict):
     return flops
 
 
-def cpu_baseline(layers, rows: int | None = None, reorder: bool = False, fp8: bool = False):
+def cpu_baseline(layers, rows: int | None = None, reorder: bool = False, fmt: str = "nvfp4"):
     """The oracle on the host cores: `rows` token rows (default two per host thread, so every
     thread works) of each layer, about 10-30 s of CPU work."""
     import oracle as O
 
     rows = rows or 2 * O._threads()
-    cache = oracle_cache(layers, max(rows, 64), reorder, fp8)
+    cache = oracle_cache(layers, max(rows, 64), reorder, fmt)
     t0 = time.perf_counter()
     flops = oracle_sample_step(layers, rows, cache)
     dt = time.perf_counter() - t0
@@ -624,7 +729,7 @@ def run_reference(args, rank, world, layers, desc):
     import oracle as O
 
     rows = O._threads()  # one token row per host thread per step
-    cache = oracle_cache(layers, max(rows, 64), getattr(args, "reorder", False), getattr(args, "format", "") == "fp8")
+    cache = oracle_cache(layers, max(rows, 64), getattr(args, "reorder", False), getattr(args, "format", "nvfp4"))
     for _ in range(args.warmup):
         oracle_sample_step(layers, rows, cache)
     t0 = time.perf_counter()
@@ -633,7 +738,8 @@ def run_reference(args, rank, world, layers, desc):
         flops += oracle_sample_step(layers, rows, cache)
     dt = time.perf_counter() - t0
     v = flops / dt / 1e12
-    metric = METRIC_FP8 if getattr(args, "format", "") == "fp8" else METRIC
+    fmt = getattr(args, "format", "nvfp4")
+    metric = METRIC_FP8 if fmt == "fp8" else METRIC_MX if fmt == "mxfp4" else METRIC
     line = {"impl": "reference", "metric": metric, "value": v, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -657,28 +763,82 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
     ap.add_argument("--proj", default="all", help="profiling: run only this layer (e.g. qkv, gateup)")
-    ap.add_argument("--format", default="nvfp4", choices=["nvfp4", "fp8"],
-                    help="linear-layer workloads: NVFP4 + ARC (default) or FP8 W8A8 with per-tensor scales")
+    ap.add_argument("--format", default="nvfp4", choices=["nvfp4", "mxfp4", "fp8"],
+                    help="linear-layer workloads: NVFP4 + ARC (default), MXFP4 + ARC (32-value blocks, "
+                         "power-of-two scales, no tensor scale) or FP8 W8A8 with per-tensor scales")
     ap.add_argument("--reorder", action="store_true",
                     help="linear-layer workloads: channels reordered by calibration abs-max before the primary "
                          "quantization (the outlier set is the first r of the order)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    if "WORLD_SIZE" in os.environ:
+        # launched by torchrun (or another launcher): one process per GPU already
+        if int(os.environ["WORLD_SIZE"]) != args.gpus:
+            ap.error(f"--gpus {args.gpus} but WORLD_SIZE={os.environ['WORLD_SIZE']}")
+        run(args, ap)
+    elif args.gpus > 1 and args.impl == "ours":
+        # no launcher: start one process per GPU here (spawned, NCCL over the visible GPUs)
+        n = torch.cuda.device_count()
+        if n < args.gpus:
+            ap.error(f"--gpus {args.gpus} but only {n} CUDA device(s) are visible")
+        spawn_ranks(args)
+    else:
+        # one GPU; or the oracle arm, which rank 0 alone runs (the other ranks have no work)
+        os.environ.setdefault("WORLD_SIZE", str(args.gpus))
+        run(args, ap)
 
+
+def _free_port() -> int:
+    import socket
+
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        return so.getsockname()[1]
+
+
+def _rank_main(local_rank: int, args, port: int):
+    os.environ.update({"RANK": str(local_rank), "LOCAL_RANK": str(local_rank), "WORLD_SIZE": str(args.gpus),
+                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    run(args, None)
+
+
+def spawn_ranks(args):
+    """One process per GPU (ranks 0..N-1 on devices 0..N-1), the same rendezvous torchrun would
+    give them; rank 0 prints the JSON line. A rank that fails makes the launch raise."""
+    import torch.multiprocessing as mp
+
+    mp.start_processes(_rank_main, args=(args, _free_port()), nprocs=args.gpus, start_method="spawn", join=True)
+
+
+def run(args, ap):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    def fail(msg):
+        if ap is not None:
+            ap.error(msg)
+        raise SystemExit(msg)
+
     layers, desc = None, None
     if args.workload != "recurrent":
         layers, desc = layer_set(args.workload)
         if args.proj != "all":
             layers = [L for L in layers if L["name"] == args.proj]
             if not layers:
-                ap.error("unknown --proj")
+                fail("unknown --proj")
+    if args.format == "mxfp4" and layers is not None:
+        if args.reorder:
+            fail("--reorder applies to the NVFP4 format")
+        for L in layers:
+            L["mx"] = True
+        desc = f"{desc}; run in MXFP4 + ARC (32-value blocks, E8M0 scales)"
     if args.format == "fp8" and layers is not None:
         if args.reorder:
-            ap.error("--reorder applies to the NVFP4 format")
+            fail("--reorder applies to the NVFP4 format")
         for L in layers:
             L["r"], L["fp8"] = 0, True
         desc = f"{desc}; run in FP8 W8A8 (per-tensor scales, no residual channels)"
@@ -701,10 +861,10 @@ def main():
             line = run_recurrent(args, rank, world, device)
         else:
             res = run_layers(args, rank, world, device, layers,
-                             with_error=args.workload == "stress" or args.reorder or args.format == "fp8")
+                             with_error=args.workload == "stress" or args.reorder or args.format != "nvfp4")
             line = layers_line(args, world, layers, desc, res) if rank == 0 else None
             if rank == 0 and not args.no_cpu_baseline:
-                line["cpu_baseline"] = cpu_baseline(layers, reorder=args.reorder, fp8=args.format == "fp8")
+                line["cpu_baseline"] = cpu_baseline(layers, reorder=args.reorder, fmt=args.format)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

@@ -240,6 +240,49 @@ arc_status arc_gemm_fp8(const uint8_t* a_codes, int64_t lda, const float* d_a_sc
                         int64_t ldy, const void* add_bf16, int64_t ld_add, arc_stream_t stream);
 
 /* ----------------------------------------------------------------------------------------- */
+/* MXFP4 with augmented residual channels ("ARCQuant", Resultaten / Generaliseerbaarheid: the    */
+/* approach extends to MXFP4)                                                                   */
+/* ----------------------------------------------------------------------------------------- */
+/*
+ * Format (this library's reading, the OCP microscaling MXFP4): 32 consecutive K-elements share
+ * one power-of-two scale X = 2^(floor(log2 amax) - 2) stored as an E8M0 byte (exponent + 127,
+ * clamped to [0, 254]; 0 for an all-zero block); elements are E2M1_rne_sat(x / X) with the sign
+ * of x kept (zero codes for an all-zero block). No tensor scale.
+ * Layouts: codes as for NVFP4, [rows, K_pad/2] with K_pad = K + r rounded up to 64. Scale bytes
+ * in 512-byte atoms of 128 rows x 4 scales (128 K-elements): the atom of rows 128i.. and scale
+ * columns 4j.. at byte (i * ceil(K_pad/128) + j) * 512, row m / column kb inside at
+ * (m%32)*16 + ((m/32)%4)*4 + kb%4; padding rows and columns are zero.
+ */
+
+/* Bytes of the MXFP4 scale layout: ceil(rows/128) * ceil(K_pad/128) * 512. */
+size_t arc_mxfp4_sf_bytes(int64_t rows, int64_t k_aug);
+
+/*
+ * Quantize bf16 X [M, K] to MXFP4 and append r residual channels: for j < r and c = d_idx[j],
+ * R[m, j] = x[m, c] - E2M1(code) * X_block(c) (exact product, fp32 subtract), coded in blocks of
+ * 32 in idx order at columns K + j. One kernel, one read of X, no workspace.
+ * Requires K % 32 == 0, r % 32 == 0, 0 <= r <= K, ldx >= K, 16-byte aligned rows and outputs.
+ * Per warp the kernel keeps K/32 + 4r bytes of shared memory (at most 200 KB in all): larger
+ * requests return ARC_ERR_UNSUPPORTED.
+ */
+arc_status arc_quantize_act_mxfp4(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, const int32_t* d_idx,
+                                  int32_t r, uint8_t* codes, uint8_t* sf, arc_stream_t stream);
+
+/* Weights W [N, K] as W_aug = [W | W[:, idx]] in MXFP4 (the r duplicated channels re-blocked
+ * among themselves in blocks of 32). Requirements as arc_quantize_act_mxfp4. */
+arc_status arc_pack_weight_mxfp4(const void* w_bf16, int64_t N, int64_t K, int64_t ldw, const int32_t* d_idx,
+                                 int32_t r, uint8_t* codes, uint8_t* sf, arc_stream_t stream);
+
+/*
+ * Y [M, N] bf16 = bf16_rn( sum_{k < K_pad} E2M1(a) X_A * E2M1(b) X_B ) [ + add ] over MXFP4
+ * operands of depth K_aug (tcgen05 kind::mxf4nvf4 with scale_vec::2X and UE8M0 scales, fp32
+ * accumulation in tensor memory). Requirements as arc_gemm_nvfp4.
+ */
+arc_status arc_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf, const uint8_t* b_codes, const uint8_t* b_sf,
+                          int64_t M, int64_t N, int64_t k_aug, void* y_bf16, int64_t ldy, const void* add_bf16,
+                          int64_t ld_add, arc_stream_t stream);
+
+/* ----------------------------------------------------------------------------------------- */
 /* Elementwise pieces of the recurrent SwiGLU block                                            */
 /* ----------------------------------------------------------------------------------------- */
 
@@ -256,10 +299,13 @@ arc_status arc_silu_mul_bf16(const void* gu_bf16, int64_t S, int64_t F, int64_t 
 /* ----------------------------------------------------------------------------------------- */
 
 /*
- * One pre-norm SwiGLU residual sublayer: h <- h + W_down (silu(W_g n) * (W_u n)), n = RMSNorm(h)*g.
- * All pointers are device pointers. The NVFP4 fields are the arc_pack_weight_nvfp4 outputs of
- * the same weights augmented with idx_gateup (channels of n, in [0, d)) and idx_down (channels
- * of the SwiGLU output, in [0, ffn)).
+ * One pre-norm SwiGLU residual sublayer: h <- beta h + W_down (silu(W_g n) * (W_u n)),
+ * n = RMSNorm(h)*g, beta = the block's residual_scale. All pointers are device pointers. The
+ * NVFP4 fields are the arc_pack_weight_nvfp4 outputs of the same weights augmented with
+ * idx_gateup (channels of n, in [0, d)) and idx_down (channels of the SwiGLU output, in
+ * [0, ffn)). The FP8 fields are the arc_quantize_fp8 outputs of the same weights (codes with row
+ * strides d and ffn bytes, and their tensor scales); they are read only by FP8 steps and may be
+ * NULL when no step runs in FP8.
  */
 typedef struct {
   const void* rms_gain_bf16;  /* [d] */
@@ -275,6 +321,10 @@ typedef struct {
   int32_t r_gateup;
   const int32_t* idx_down;
   int32_t r_down;
+  const uint8_t* gateup_fp8;      /* [2*ffn, d] E4M3 */
+  const float* gateup_fp8_scale;
+  const uint8_t* down_fp8;        /* [d, ffn] E4M3 */
+  const float* down_fp8_scale;
 } arc_swiglu_sublayer;
 
 typedef struct {
@@ -283,6 +333,9 @@ typedef struct {
   float eps;      /* RMSNorm epsilon */
   int32_t n_sublayers;
   const arc_swiglu_sublayer* sublayers; /* host array of n_sublayers entries */
+  float residual_scale; /* beta in (0, 1] of the damped residual h <- beta h + F(h); 0 or 1 is the
+                           plain residual block. beta < 1 makes the step map contractive when F
+                           is small, the regime of RAMP's error analysis (section 3). */
 } arc_swiglu_block;
 
 /* Workspace of arc_recurrent_prefill for S tokens. */
@@ -301,10 +354,19 @@ arc_status arc_recurrent_prefill(void* h_bf16, int64_t S, const arc_swiglu_block
 /*
  * The same recurrence with any per-step precision schedule (for schedule studies: RAMP's
  * matched-budget comparison of where the BF16 steps go, "RAMP…" §6 and its Early-BF16 and
- * random-schedule baselines): low_steps is a host array of T bytes, read during the call;
- * step t runs in NVFP4 + ARC when low_steps[t] != 0, else in BF16. arc_recurrent_prefill with
- * k_low is the schedule low_steps[t] = (t < k_low).
+ * random-schedule baselines; and RAMP's own FP8-BF16 instantiation, §4.2): low_steps is a host
+ * array of T bytes, read during the call, one format per step:
+ *   ARC_STEP_BF16 (0)   BF16 (RMSNorm, BF16 GEMMs);
+ *   ARC_STEP_NVFP4 (1)  NVFP4 + ARC (as arc_recurrent_prefill's steps before k_low);
+ *   ARC_STEP_FP8 (2)    FP8 W8A8 with per-tensor scales: RMSNorm, arc_quantize_fp8 (dynamic
+ *                       scale), arc_gemm_fp8 with the sublayer's FP8 weights, SwiGLU,
+ *                       arc_quantize_fp8, arc_gemm_fp8 with the residual add.
+ * Any other value, or an FP8 step with NULL FP8 weights, returns ARC_ERR_INVALID_ARG before any
+ * launch. arc_recurrent_prefill with k_low is the schedule low_steps[t] = (t < k_low).
  */
+#define ARC_STEP_BF16 0
+#define ARC_STEP_NVFP4 1
+#define ARC_STEP_FP8 2
 arc_status arc_recurrent_prefill_schedule(void* h_bf16, int64_t S, const arc_swiglu_block* blk, int32_t T,
                                           const uint8_t* low_steps, void* workspace, size_t ws_bytes,
                                           arc_stream_t stream);

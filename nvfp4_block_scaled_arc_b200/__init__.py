@@ -36,12 +36,18 @@ class SwigluSublayer(ctypes.Structure):
         ("down_codes", ctypes.c_void_p), ("down_sf", ctypes.c_void_p), ("down_scale", ctypes.c_void_p),
         ("idx_gateup", ctypes.c_void_p), ("r_gateup", ctypes.c_int32),
         ("idx_down", ctypes.c_void_p), ("r_down", ctypes.c_int32),
+        ("gateup_fp8", ctypes.c_void_p), ("gateup_fp8_scale", ctypes.c_void_p),
+        ("down_fp8", ctypes.c_void_p), ("down_fp8_scale", ctypes.c_void_p),
     ]
 
 
 class SwigluBlock(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int64), ("ffn", ctypes.c_int64), ("eps", ctypes.c_float),
-                ("n_sublayers", ctypes.c_int32), ("sublayers", ctypes.POINTER(SwigluSublayer))]
+                ("n_sublayers", ctypes.c_int32), ("sublayers", ctypes.POINTER(SwigluSublayer)),
+                ("residual_scale", ctypes.c_float)]
+
+
+STEP_BF16, STEP_NVFP4, STEP_FP8 = 0, 1, 2  # per-step formats of arc_recurrent_prefill_schedule
 
 
 _SIGS = {
@@ -76,6 +82,16 @@ _SIGS = {
                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                       ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64,
                                       ctypes.c_void_p]),
+    "arc_mxfp4_sf_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64]),
+    "arc_quantize_act_mxfp4": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                              ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                                              ctypes.c_void_p]),
+    "arc_pack_weight_mxfp4": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                             ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                                             ctypes.c_void_p]),
+    "arc_gemm_mxfp4": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                      ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64,
+                                      ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]),
     "arc_gemm_bf16": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                                      ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                      ctypes.c_int64, ctypes.c_void_p]),
@@ -332,20 +348,26 @@ def silu_mul_bf16(gu: torch.Tensor, out: torch.Tensor | None = None, stream=None
 
 
 class RecurrentBlock:
-    """Host description of the shared SwiGLU block (keeps the ctypes structs and tensors alive)."""
+    """Host description of the shared SwiGLU block (keeps the ctypes structs and tensors alive).
+    Each sublayer dict holds gain, wgu, wd (bf16), gu_q, d_q (packed NVFP4 weights), idx_gu,
+    idx_d, and optionally gu_f8, d_f8 (FP8Tensor weights, needed by FP8 steps).
+    residual_scale is the damped residual's beta (1: the plain residual block)."""
 
-    def __init__(self, d: int, ffn: int, eps: float, sublayers: list[dict]):
+    def __init__(self, d: int, ffn: int, eps: float, sublayers: list[dict], residual_scale: float = 1.0):
         self.d, self.ffn, self.eps = d, ffn, eps
         self.sub = sublayers
         arr = (SwigluSublayer * len(sublayers))()
         for i, L in enumerate(sublayers):
+            f8g, f8d = L.get("gu_f8"), L.get("d_f8")
             arr[i] = SwigluSublayer(
                 L["gain"].data_ptr(), L["wgu"].data_ptr(), L["wd"].data_ptr(),
                 L["gu_q"].codes.data_ptr(), L["gu_q"].sf.data_ptr(), L["gu_q"].scale.data_ptr(),
                 L["d_q"].codes.data_ptr(), L["d_q"].sf.data_ptr(), L["d_q"].scale.data_ptr(),
-                L["idx_gu"].data_ptr(), int(L["idx_gu"].numel()), L["idx_d"].data_ptr(), int(L["idx_d"].numel()))
+                L["idx_gu"].data_ptr(), int(L["idx_gu"].numel()), L["idx_d"].data_ptr(), int(L["idx_d"].numel()),
+                f8g.codes.data_ptr() if f8g is not None else None, f8g.scale.data_ptr() if f8g is not None else None,
+                f8d.codes.data_ptr() if f8d is not None else None, f8d.scale.data_ptr() if f8d is not None else None)
         self._arr = arr
-        self.block = SwigluBlock(d, ffn, float(eps), len(sublayers), arr)
+        self.block = SwigluBlock(d, ffn, float(eps), len(sublayers), arr, float(residual_scale))
 
     def workspace_bytes(self, S: int) -> int:
         return int(lib().arc_recurrent_workspace_bytes(S, ctypes.byref(self.block)))
@@ -366,9 +388,9 @@ def recurrent_prefill(h: torch.Tensor, block: RecurrentBlock, T: int, k_low: int
 def recurrent_prefill_schedule(h: torch.Tensor, block: RecurrentBlock, schedule, workspace: torch.Tensor | None = None,
                                stream=None) -> torch.Tensor:
     """arc_recurrent_prefill_schedule: apply the block len(schedule) times in place; step t in
-    NVFP4 + ARC when schedule[t] is true, else in BF16."""
+    the format schedule[t]: STEP_BF16 (0 / False), STEP_NVFP4 (1 / True) or STEP_FP8 (2)."""
     S = h.shape[0]
-    flags = (ctypes.c_uint8 * max(1, len(schedule)))(*[1 if f else 0 for f in schedule])
+    flags = (ctypes.c_uint8 * max(1, len(schedule)))(*[int(f) for f in schedule])
     n = block.workspace_bytes(S)
     if workspace is None:
         workspace = _ws(n, h.device)
@@ -376,6 +398,64 @@ def recurrent_prefill_schedule(h: torch.Tensor, block: RecurrentBlock, schedule,
         _p(h), S, ctypes.byref(block.block), len(schedule), flags, _p(workspace), workspace.numel(),
         _stream(stream)))
     return h
+
+
+@dataclass
+class MXFP4Tensor:
+    """Packed MXFP4 operand: codes [rows, K_pad/2] u8 and swizzled E8M0 scale bytes (no tensor scale)."""
+    codes: torch.Tensor
+    sf: torch.Tensor
+    rows: int
+    k_aug: int
+
+
+def mxfp4_sf_bytes(rows: int, k_aug: int) -> int:
+    return int(lib().arc_mxfp4_sf_bytes(rows, k_aug))
+
+
+def _mx_out(rows, k_aug, device):
+    return MXFP4Tensor(_u8(codes_bytes(rows, k_aug), device), _u8(mxfp4_sf_bytes(rows, k_aug), device), rows, k_aug)
+
+
+def quantize_act_mxfp4(x: torch.Tensor, idx: torch.Tensor | None = None, out: MXFP4Tensor | None = None,
+                       stream=None) -> MXFP4Tensor:
+    """arc_quantize_act_mxfp4: X [M, K] bf16 -> MXFP4 with r appended residual channels."""
+    _need_cuda(x, idx)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    M, K = x.shape
+    r = 0 if idx is None else int(idx.numel())
+    if out is None:
+        out = _mx_out(M, K + r, x.device)
+    _check("arc_quantize_act_mxfp4", lib().arc_quantize_act_mxfp4(_p(x), M, K, x.stride(0), _p(idx), r, _p(out.codes),
+                                                                  _p(out.sf), _stream(stream)))
+    return out
+
+
+def pack_weight_mxfp4(w: torch.Tensor, idx: torch.Tensor | None = None, out: MXFP4Tensor | None = None,
+                      stream=None) -> MXFP4Tensor:
+    """arc_pack_weight_mxfp4: W [N, K] bf16 -> W_aug = [W | W[:, idx]] in MXFP4."""
+    _need_cuda(w, idx)
+    assert w.dtype == torch.bfloat16 and w.dim() == 2 and w.stride(1) == 1
+    N, K = w.shape
+    r = 0 if idx is None else int(idx.numel())
+    if out is None:
+        out = _mx_out(N, K + r, w.device)
+    _check("arc_pack_weight_mxfp4", lib().arc_pack_weight_mxfp4(_p(w), N, K, w.stride(0), _p(idx), r, _p(out.codes),
+                                                                _p(out.sf), _stream(stream)))
+    return out
+
+
+def gemm_mxfp4(a: MXFP4Tensor, b: MXFP4Tensor, out: torch.Tensor | None = None, add: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """arc_gemm_mxfp4: Y [M, N] bf16 = MXFP4(A) MXFP4(B)^T over depth K_aug (+ add)."""
+    assert a.k_aug == b.k_aug
+    M, N = a.rows, b.rows
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=a.codes.device)
+    _check("arc_gemm_mxfp4", lib().arc_gemm_mxfp4(
+        _p(a.codes), _p(a.sf), _p(b.codes), _p(b.sf), M, N, a.k_aug, _p(out), out.stride(0), _p(add),
+        0 if add is None else add.stride(0), _stream(stream)))
+    return out
 
 
 class FP8Tensor:

@@ -184,6 +184,20 @@ __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uin
       : "memory");
 }
 
+// D (+)= A B^T with E2M1 A and B and one UE8M0 scale per 32 elements of each (MXFP4): the same
+// instruction with scale_vec::2X, the two scales of a row's K = 64 step in bytes 0 and 1 of its
+// tensor-memory scale cell.
+__device__ __forceinline__ void tc_mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
 // Instruction descriptors (dense, K-major A and B, fp32 accumulate).
 //   bf16:  c=f32 (bits 4-5), a=bf16 (7-9), b=bf16 (10-12), N>>3 (17-22), M>>4 (24-28)
 //   nvf4:  a=b=E2M1 (value 1), scale type UE4M3 (bit 23 = 0), scale-factor ids 0, K = 64
@@ -198,6 +212,8 @@ __host__ __device__ constexpr uint32_t idesc_f8(int M, int N) {
 __host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
   return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
+//   mxf4:  as nvf4 with scale type UE8M0 (bit 23 = 1)
+__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N) { return idesc_nvf4(M, N) | (1u << 23); }
 
 // 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives lane (base + i).
 __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {

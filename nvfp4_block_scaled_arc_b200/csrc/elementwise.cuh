@@ -60,6 +60,26 @@ __global__ void __launch_bounds__(256) k_silu_mul(const __nv_bfloat16* __restric
   }
 }
 
+// h[m, k] = bf16(beta * h[m, k]) in place, 8 values per thread (d % 8 == 0): the damped residual
+// of a contractive recurrent block, applied before the sublayer's residual add.
+__global__ void __launch_bounds__(256) k_scale_bf16(__nv_bfloat16* __restrict__ h, int64_t ldh, int M, int d,
+                                                    float beta) {
+  const int vpr = d >> 3;
+  const int64_t total = static_cast<int64_t>(M) * vpr;
+  for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < total;
+       v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = v / vpr;
+    const int j = static_cast<int>(v - m * vpr) * 8;
+    uint4* p = reinterpret_cast<uint4*>(h + m * ldh + j);
+    const uint4 w = *p;
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = pack_bf16x2_rn(__fmul_rn(beta, bf16_lo(ws[i])), __fmul_rn(beta, bf16_hi(ws[i])));
+    *p = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
 // Per-channel max |x| over rows (fp32 bit patterns, atomicMax), channel pairs per thread.
 __global__ void __launch_bounds__(256) k_colmax(const __nv_bfloat16* __restrict__ x, int64_t ldx, int M, int K,
                                                 int rows_per_cta, uint32_t* colmax) {

@@ -46,7 +46,7 @@
 namespace arc {
 
 // GEMM kinds: the BF16 reference GEMM, the block-scaled NVFP4 GEMM, the per-tensor-scaled FP8 GEMM.
-constexpr int kGemmBF16 = 0, kGemmFP4 = 1, kGemmFP8 = 2;
+constexpr int kGemmBF16 = 0, kGemmFP4 = 1, kGemmFP8 = 2, kGemmMX4 = 3;
 
 template <int KIND>
 struct GemmTraits;
@@ -71,6 +71,19 @@ struct GemmTraits<kGemmBF16> {
   static constexpr uint32_t IDESC = idesc_bf16(BM, BN);
   static constexpr int TMEM_COLS = 512;
   static constexpr int SF_COL0 = 0, SF_SET_COLS = 0;
+};
+
+// MXFP4: the FP4 geometry with one UE8M0 scale per 32 elements; a stage's 256 K-elements per row
+// are 8 scales, two 512-byte atoms per 128-row block.
+template <>
+struct GemmTraits<kGemmMX4> {
+  static constexpr int BM = 128, BN = 256, STAGES = 4, ACC_STAGES = 1;
+  static constexpr int A_BYTES = BM * 128, B_BYTES = BN * 128;
+  static constexpr int SFA_BYTES = 2 * 512, SFB_BYTES = 2 * 2 * 512;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr uint32_t IDESC = idesc_mxf4(BM, BN);
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int SF_COL0 = 256, SF_SET_COLS = 64;
 };
 
 // FP8: the BF16 geometry (128 bytes of K per row and stage = 128 E4M3 values, 4 MMAs of K = 32)
@@ -155,7 +168,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
            const __grid_constant__ CUtensorMap tmY, const GemmArgs g) {
   using T = GemmTraits<KIND>;
-  constexpr bool FP4 = KIND == kGemmFP4, FP8 = KIND == kGemmFP8;
+  constexpr bool NV4 = KIND == kGemmFP4, MX4 = KIND == kGemmMX4, FP8 = KIND == kGemmFP8;
+  constexpr bool FP4 = NV4 || MX4;  // block-scaled E2M1 operands, scales in tensor memory
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + T::STAGES * T::STAGE_BYTES;  // 8 x 1 KB, one per epilogue warp
@@ -217,8 +231,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           } else {
             uint32_t bytes = static_cast<uint32_t>(g.box_rows_a + g.box_rows_b) * 128u;
             int natoms = 0, nb = 0;
+            constexpr int APS = MX4 ? 2 : 4;  // scale atoms per stage and 128-row block
             if (FP4) {
-              natoms = min(4, g.katoms - 4 * ks);
+              natoms = min(APS, g.katoms - APS * ks);
               nb = min(2, g.nblk128 - 2 * tn);
               bytes += static_cast<uint32_t>(natoms * 512 * (1 + nb));
             }
@@ -229,9 +244,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (FP4) {
               uint8_t* sSFA = sB + T::B_BYTES;
               uint8_t* sSFB = sSFA + T::SFA_BYTES;
-              bulk_load(sSFA, g.sfa + (static_cast<int64_t>(tm) * g.katoms + 4 * ks) * 512, natoms * 512, &full[stage]);
+              bulk_load(sSFA, g.sfa + (static_cast<int64_t>(tm) * g.katoms + APS * ks) * 512, natoms * 512, &full[stage]);
               for (int b = 0; b < nb; ++b)
-                bulk_load(sSFB + b * 2048, g.sfb + (static_cast<int64_t>(2 * tn + b) * g.katoms + 4 * ks) * 512,
+                bulk_load(sSFB + b * APS * 512, g.sfb + (static_cast<int64_t>(2 * tn + b) * g.katoms + APS * ks) * 512,
                           natoms * 512, &full[stage]);
             }
             armed |= 1u << stage;
@@ -268,15 +283,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_after();
           uint8_t* sA = smem + stage * T::STAGE_BYTES;
           uint8_t* sB = sA + T::A_BYTES;
-          const int nk = (FP4 || FP8) ? min(4, g.ksteps - 4 * ks) : 4;
+          const int nk = (FP4 || FP8) ? min(4, g.ksteps - 4 * ks) : 4;  // MMAs in this stage
           const uint64_t da = desc_kmajor_sw128(smem_u32(sA));
           const uint64_t db = desc_kmajor_sw128(smem_u32(sB));
           const uint32_t sf = tmem + T::SF_COL0 + T::SF_SET_COLS * stage;
           for (int k = 0; k < nk; ++k) {
             const uint64_t off = static_cast<uint64_t>((k * 32) >> 4);
             const uint32_t accum = (ks > 0 || k > 0) ? 1u : 0u;
-            if (FP4)
+            if (NV4)
               tc_mma_nvf4(d_tmem, da + off, db + off, T::IDESC, sf + 32 + 4 * k, sf + 8 * k, accum);
+            else if (MX4)
+              tc_mma_mxf4(d_tmem, da + off, db + off, T::IDESC, sf + 32 + 4 * k, sf + 8 * k, accum);
             else if (FP8)
               tc_mma_f8(d_tmem, da + off, db + off, T::IDESC, accum);
             else
@@ -316,26 +333,53 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           tc_fence_after();
-          const int natoms = min(4, g.katoms - 4 * ks);
           const uint32_t sSFA = smem_u32(smem + stage * T::STAGE_BYTES + T::A_BYTES + T::B_BYTES);
           const uint32_t sSFB = sSFA + T::SFA_BYTES;
-          uint32_t v[32];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            uint4 b0 = make_uint4(0, 0, 0, 0), b1 = b0;
-            if (k < natoms) {
-              b0 = lds_u32x4(sSFB + k * 512 + lane * 16);
-              b1 = lds_u32x4(sSFB + 2048 + k * 512 + lane * 16);
-            }
-            v[8 * k + 0] = b0.x, v[8 * k + 1] = b0.y, v[8 * k + 2] = b0.z, v[8 * k + 3] = b0.w;
-            v[8 * k + 4] = b1.x, v[8 * k + 5] = b1.y, v[8 * k + 6] = b1.z, v[8 * k + 7] = b1.w;
-          }
           const uint32_t set = lane_base + T::SF_COL0 + T::SF_SET_COLS * stage;
-          tmem_st_32x32b_x32(set, v);
+          uint32_t v[32];
+          if (NV4) {
+            // one atom per K = 64 step: a row's 4 scales are one 32-bit cell
+            const int natoms = min(4, g.katoms - 4 * ks);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t a = (k < natoms) ? lds_u32(sSFA + k * 512 + lane * 16 + 4 * q) : 0u;
-            tmem_st_32x32b_x1(set + 32 + 4 * k + q, a);
+            for (int k = 0; k < 4; ++k) {
+              uint4 b0 = make_uint4(0, 0, 0, 0), b1 = b0;
+              if (k < natoms) {
+                b0 = lds_u32x4(sSFB + k * 512 + lane * 16);
+                b1 = lds_u32x4(sSFB + 2048 + k * 512 + lane * 16);
+              }
+              v[8 * k + 0] = b0.x, v[8 * k + 1] = b0.y, v[8 * k + 2] = b0.z, v[8 * k + 3] = b0.w;
+              v[8 * k + 4] = b1.x, v[8 * k + 5] = b1.y, v[8 * k + 6] = b1.z, v[8 * k + 7] = b1.w;
+            }
+            tmem_st_32x32b_x32(set, v);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint32_t a = (k < natoms) ? lds_u32(sSFA + k * 512 + lane * 16 + 4 * q) : 0u;
+              tmem_st_32x32b_x1(set + 32 + 4 * k + q, a);
+            }
+          } else {
+            // MXFP4: one atom per two K = 64 steps; step k's two scales are half k % 2 of the
+            // atom's 32-bit word, stored in bytes 0 and 1 of the step's cell
+            const int natoms = min(2, g.katoms - 2 * ks);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int at = k >> 1, sh = 16 * (k & 1);
+              uint4 b0 = make_uint4(0, 0, 0, 0), b1 = b0;
+              if (at < natoms) {
+                b0 = lds_u32x4(sSFB + at * 512 + lane * 16);
+                b1 = lds_u32x4(sSFB + 1024 + at * 512 + lane * 16);
+              }
+              v[8 * k + 0] = (b0.x >> sh) & 0xFFFFu, v[8 * k + 1] = (b0.y >> sh) & 0xFFFFu;
+              v[8 * k + 2] = (b0.z >> sh) & 0xFFFFu, v[8 * k + 3] = (b0.w >> sh) & 0xFFFFu;
+              v[8 * k + 4] = (b1.x >> sh) & 0xFFFFu, v[8 * k + 5] = (b1.y >> sh) & 0xFFFFu;
+              v[8 * k + 6] = (b1.z >> sh) & 0xFFFFu, v[8 * k + 7] = (b1.w >> sh) & 0xFFFFu;
+            }
+            tmem_st_32x32b_x32(set, v);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int at = k >> 1, sh = 16 * (k & 1);
+              const uint32_t a = (at < natoms) ? (lds_u32(sSFA + at * 512 + lane * 16 + 4 * q) >> sh) & 0xFFFFu : 0u;
+              tmem_st_32x32b_x1(set + 32 + 4 * k + q, a);
+            }
           }
           tmem_st_wait();
           tc_fence_before();
@@ -357,7 +401,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // stored 32 columns at a time.
     const int q = warp & 3;
     const int half = (warp - kGemmEpiWarp0) >> 2;
-    const float alpha = (FP4 || FP8) ? __fmul_rn(*g.a_scale, *g.b_scale) : 1.0f;
+    const float alpha = (NV4 || FP8) ? __fmul_rn(*g.a_scale, *g.b_scale) : 1.0f;  // MXFP4: no tensor scales
     const uint64_t alpha2 = f2_pack(alpha, alpha);
     constexpr int HB = T::BN / 2;  // columns per warp
     uint32_t acc = 0, acc_phase = 0;

@@ -64,6 +64,12 @@ arc_status device_check(int* sms) {
                              arc::kQRowsSmemMax) != cudaSuccess ||
         cudaFuncSetAttribute(arc::k_quant_rows<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              arc::kQRowsSmemMax) != cudaSuccess ||
+        cudaFuncSetAttribute(arc::k_gemm<arc::kGemmMX4, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             arc::gemm_smem_bytes<arc::kGemmMX4>()) != cudaSuccess ||
+        cudaFuncSetAttribute(arc::k_gemm<arc::kGemmMX4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             arc::gemm_smem_bytes<arc::kGemmMX4>()) != cudaSuccess ||
+        cudaFuncSetAttribute(arc::k_quant_mx_rows, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             arc::kQRowsSmemMax) != cudaSuccess ||
         cudaFuncSetAttribute(arc::k_quant_reordered<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              arc::kQReoSmemMax) != cudaSuccess ||
         cudaFuncSetAttribute(arc::k_quant_reordered<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -165,8 +171,9 @@ arc_status quantize_check(const void* x, int64_t M, int64_t K, int64_t ldx, cons
   if (M <= 0 || K <= 0 || K % 16 || r < 0 || r % 16 || r > K || ldx < K) return ARC_ERR_INVALID_ARG;
   if (!perm && r > 0 && !idx) return ARC_ERR_INVALID_ARG;
   if (M > (1ll << 30) || K > (1ll << 20) || r > 32767) return ARC_ERR_UNSUPPORTED;
-  const size_t smem = perm ? arc::qreo_smem_bytes(static_cast<int>(K)) : arc::qrows_smem_bytes(static_cast<int>(K), r);
-  if (smem > static_cast<size_t>(perm ? arc::kQReoSmemMax : arc::kQRowsSmemMax)) return ARC_ERR_UNSUPPORTED;
+  if (perm ? arc::qreo_smem_bytes(static_cast<int>(K)) > static_cast<size_t>(arc::kQReoSmemMax)
+           : arc::qrows_warps(static_cast<int>(K), r) < 1)
+    return ARC_ERR_UNSUPPORTED;
   if (!al16(x) || (ldx * 2) % 16 || !al16(codes) || !al16(sf) || (gain && !al16(gain)) || (perm && !al16(perm)))
     return ARC_ERR_ALIGNMENT;
   return ARC_OK;
@@ -178,7 +185,9 @@ arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, con
                            const int32_t* perm = nullptr) {
   arc_status st = quantize_check(x, M, K, ldx, idx, r, gain, codes, sf, scale_out, perm);
   if (st != ARC_OK) return st;
-  const size_t smem = perm ? arc::qreo_smem_bytes(static_cast<int>(K)) : arc::qrows_smem_bytes(static_cast<int>(K), r);
+  const int qwarps = arc::qrows_warps(static_cast<int>(K), r);
+  const size_t smem = perm ? arc::qreo_smem_bytes(static_cast<int>(K))
+                           : arc::qrows_smem_bytes(static_cast<int>(K), r, qwarps);
   if (!workspace || ws_bytes < arc_quantize_workspace_bytes(M, r)) return ARC_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ARC_ERR_ALIGNMENT;
   int sms = 0;
@@ -253,18 +262,18 @@ arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, con
   const void* kern = gain ? reinterpret_cast<const void*>(arc::k_quant_rows<true>)
                           : reinterpret_cast<const void*>(arc::k_quant_rows<false>);
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, arc::kQRowThreads, smem) != cudaSuccess ||
-      per_sm < 1)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, qwarps * 32, smem) != cudaSuccess || per_sm < 1)
     return ARC_ERR_CUDA;
-  const int64_t want = mpad;  // one row per CTA at a time
-  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(want, static_cast<int64_t>(sms) * per_sm));
+  // one warp per row at a time, rows dealt round-robin over one resident wave of CTAs (every SM
+  // then holds the same number of rows to within one per CTA)
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(mpad, static_cast<int64_t>(sms) * per_sm));
   // the second launch may begin while the first one runs; it waits for the first one's results
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(arc::kQRowThreads);
+  cfg.blockDim = dim3(static_cast<unsigned>(qwarps * 32));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cfg.attrs = attr;
@@ -272,6 +281,41 @@ arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, con
   const cudaError_t e = gain ? cudaLaunchKernelEx(&cfg, arc::k_quant_rows<true>, a, mpad)
                              : cudaLaunchKernelEx(&cfg, arc::k_quant_rows<false>, a, mpad);
   return e == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
+}
+
+// MXFP4 quantization driver (activations: residuals appended; weights: channels duplicated).
+arc_status quantize_mx(const void* x, int64_t M, int64_t K, int64_t ldx, const int32_t* idx, int32_t r,
+                       uint8_t* codes, uint8_t* sf, arc_stream_t stream, int dup) {
+  if (!x || !codes || !sf) return ARC_ERR_INVALID_ARG;
+  if (M <= 0 || K <= 0 || K % 32 || r < 0 || r % 32 || r > K || ldx < K || (r > 0 && !idx)) return ARC_ERR_INVALID_ARG;
+  if (M > (1ll << 30) || K > (1ll << 20) || r > 32767) return ARC_ERR_UNSUPPORTED;
+  const int warps = arc::qmx_warps(static_cast<int>(K), r);
+  if (warps < 1) return ARC_ERR_UNSUPPORTED;
+  if (!al16(x) || (ldx * 2) % 16 || !al16(codes) || !al16(sf)) return ARC_ERR_ALIGNMENT;
+  int sms = 0;
+  arc_status st = device_check(&sms);
+  if (st != ARC_OK) return st;
+  const size_t smem = arc::qmx_smem_bytes(static_cast<int>(K), r, warps);
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, arc::k_quant_mx_rows, warps * 32, smem) != cudaSuccess ||
+      per_sm < 1)
+    return ARC_ERR_CUDA;
+  arc::QuantMxArgs a;
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  a.ldx = ldx;
+  a.M = static_cast<int>(M);
+  a.K = static_cast<int>(K);
+  a.r = r;
+  a.kpad = static_cast<int>(arc_kpad(K + r));
+  a.katoms = (a.kpad + 127) / 128;
+  a.idx = idx;
+  a.codes = codes;
+  a.sf = sf;
+  a.dup = dup;
+  const int mpad = static_cast<int>((M + 127) / 128 * 128);
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(mpad, static_cast<int64_t>(sms) * per_sm));
+  arc::k_quant_mx_rows<<<grid, warps * 32, smem, S(stream)>>>(a, mpad);
+  return launch_status();
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -327,6 +371,11 @@ size_t arc_nvfp4_codes_bytes(int64_t rows, int64_t k_aug) {
 size_t arc_nvfp4_sf_bytes(int64_t rows, int64_t k_aug) {
   if (rows <= 0 || k_aug <= 0) return 0;
   return static_cast<size_t>((rows + 127) / 128) * static_cast<size_t>(arc_kpad(k_aug) / 64) * 512u;
+}
+
+size_t arc_mxfp4_sf_bytes(int64_t rows, int64_t k_aug) {
+  if (rows <= 0 || k_aug <= 0) return 0;
+  return static_cast<size_t>((rows + 127) / 128) * static_cast<size_t>((arc_kpad(k_aug) + 127) / 128) * 512u;
 }
 
 size_t arc_quantize_workspace_bytes(int64_t rows, int32_t r) {
@@ -463,6 +512,59 @@ arc_status arc_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_sf, const flo
     return ARC_ERR_CUDA;
   g.inject = take_inject();
   return gemm_launch<arc::kGemmFP4>(ta, tb, g, sms, add_bf16 != nullptr, S(stream));
+}
+
+arc_status arc_quantize_act_mxfp4(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, const int32_t* d_idx,
+                                  int32_t r, uint8_t* codes, uint8_t* sf, arc_stream_t stream) {
+  return quantize_mx(x_bf16, M, K, ldx, d_idx, r, codes, sf, stream, 0);
+}
+
+arc_status arc_pack_weight_mxfp4(const void* w_bf16, int64_t N, int64_t K, int64_t ldw, const int32_t* d_idx,
+                                 int32_t r, uint8_t* codes, uint8_t* sf, arc_stream_t stream) {
+  return quantize_mx(w_bf16, N, K, ldw, d_idx, r, codes, sf, stream, 1);
+}
+
+arc_status arc_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf, const uint8_t* b_codes, const uint8_t* b_sf,
+                          int64_t M, int64_t N, int64_t k_aug, void* y_bf16, int64_t ldy, const void* add_bf16,
+                          int64_t ld_add, arc_stream_t stream) {
+  if (!a_codes || !a_sf || !b_codes || !b_sf || !y_bf16) return ARC_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || k_aug <= 0 || N % 8 || ldy < N || ldy % 8) return ARC_ERR_INVALID_ARG;
+  if (add_bf16 && (ld_add < N || ld_add % 8)) return ARC_ERR_INVALID_ARG;
+  if (M > (1ll << 30) || N > (1ll << 30) || k_aug > (1ll << 24)) return ARC_ERR_UNSUPPORTED;
+  if (!al16(a_codes) || !al16(a_sf) || !al16(b_codes) || !al16(b_sf) || !al16(y_bf16) ||
+      (add_bf16 && !al16(add_bf16)))
+    return ARC_ERR_ALIGNMENT;
+  int sms = 0;
+  arc_status st = device_check(&sms);
+  if (st != ARC_OK) return st;
+  const int64_t kpad = arc_kpad(k_aug);
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  g.M = static_cast<int>(M);
+  g.N = static_cast<int>(N);
+  g.ksteps = static_cast<int>(kpad / 64);
+  g.kstages = (g.ksteps + 3) / 4;
+  g.katoms = static_cast<int>((kpad + 127) / 128);
+  g.nblk128 = static_cast<int>((N + 127) / 128);
+  g.tiles_m = static_cast<int>((M + 127) / 128);
+  g.tiles_n = static_cast<int>((N + 255) / 256);
+  g.box_rows_a = static_cast<int>(std::min<int64_t>(128, M));
+  g.box_rows_b = static_cast<int>(std::min<int64_t>(256, N));
+  g.sfa = a_sf;
+  g.sfb = b_sf;
+  g.y = static_cast<__nv_bfloat16*>(y_bf16);
+  g.ldy = ldy;
+  g.add = static_cast<const __nv_bfloat16*>(add_bf16);
+  g.ld_add = ld_add;
+  g.wait_ns = g_wait_ns;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, static_cast<uint64_t>(kpad / 2),
+                static_cast<uint64_t>(M), static_cast<uint64_t>(kpad / 2), 128, g.box_rows_a) ||
+      !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b_codes, static_cast<uint64_t>(kpad / 2),
+                static_cast<uint64_t>(N), static_cast<uint64_t>(kpad / 2), 128, g.box_rows_b))
+    return ARC_ERR_CUDA;
+  g.inject = take_inject();
+  return gemm_launch<arc::kGemmMX4>(ta, tb, g, sms, add_bf16 != nullptr, S(stream));
 }
 
 arc_status arc_gemm_bf16(const void* x_bf16, int64_t ldx, const void* w_bf16, int64_t ldw, int64_t M, int64_t N,
@@ -611,7 +713,7 @@ arc_status arc_silu_mul_bf16(const void* gu_bf16, int64_t S_, int64_t F, int64_t
   return launch_status();
 }
 
-// Workspace of the recurrent driver: activation codes/scales (the larger of the two
+// Workspace of the recurrent driver: activation codes/scales (the larger of the NVFP4 and FP8
 // quantizations), two tensor scales, gate|up output, SwiGLU output, normed hidden state,
 // quantizer workspace.
 static void recurrent_layout(int64_t S_, const arc_swiglu_block* blk, size_t off[7]) {
@@ -620,7 +722,8 @@ static void recurrent_layout(int64_t S_, const arc_swiglu_block* blk, size_t off
     rmax_gu = std::max(rmax_gu, blk->sublayers[i].r_gateup);
     rmax_d = std::max(rmax_d, blk->sublayers[i].r_down);
   }
-  const size_t codes = std::max(arc_nvfp4_codes_bytes(S_, blk->d + rmax_gu), arc_nvfp4_codes_bytes(S_, blk->ffn + rmax_d));
+  const size_t codes = std::max({arc_nvfp4_codes_bytes(S_, blk->d + rmax_gu), arc_nvfp4_codes_bytes(S_, blk->ffn + rmax_d),
+                                 static_cast<size_t>(S_) * static_cast<size_t>(std::max(blk->d, blk->ffn))});
   const size_t sf = std::max(arc_nvfp4_sf_bytes(S_, blk->d + rmax_gu), arc_nvfp4_sf_bytes(S_, blk->ffn + rmax_d));
   auto a256 = [](size_t x) { return (x + 255) / 256 * 256; };
   off[0] = 0;                                                       // codes
@@ -642,14 +745,40 @@ size_t arc_recurrent_workspace_bytes(int64_t S_, const arc_swiglu_block* blk) {
   return off[6] + arc_quantize_workspace_bytes(S_, rmax);
 }
 
-// The recurrence with a per-step precision: step t runs in NVFP4 + ARC when low(t), else in BF16.
+// h = bf16(beta * h), the damped residual of a contractive block.
+static arc_status scale_bf16(void* h, int64_t S_, int64_t d, float beta, arc_stream_t stream, int sms) {
+  const int64_t vecs = S_ * (d / 8);
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((vecs + 255) / 256, static_cast<int64_t>(sms) * 8));
+  arc::k_scale_bf16<<<static_cast<unsigned>(blocks), 256, 0, S(stream)>>>(static_cast<__nv_bfloat16*>(h), d,
+                                                                         static_cast<int>(S_), static_cast<int>(d), beta);
+  return launch_status();
+}
+
+// The recurrence with a per-step format: step t runs as fmt(t) (ARC_STEP_BF16, ARC_STEP_NVFP4 or
+// ARC_STEP_FP8).
 extern "C++" {
-template <class Low>
-arc_status recurrent_run(void* h_bf16, int64_t S_, const arc_swiglu_block* blk, int32_t T, Low low_step,
+template <class Fmt>
+arc_status recurrent_run(void* h_bf16, int64_t S_, const arc_swiglu_block* blk, int32_t T, Fmt fmt,
                          void* workspace, size_t ws_bytes, arc_stream_t stream) {
   if (!h_bf16 || !blk || !blk->sublayers || blk->n_sublayers <= 0 || S_ <= 0 || T < 0) return ARC_ERR_INVALID_ARG;
   const int64_t d = blk->d, F = blk->ffn;
   if (d <= 0 || F <= 0 || d % 16 || F % 16) return ARC_ERR_INVALID_ARG;
+  const float beta = blk->residual_scale == 0.0f ? 1.0f : blk->residual_scale;
+  if (!(beta > 0.0f && beta <= 1.0f)) return ARC_ERR_INVALID_ARG;
+  for (int32_t t = 0; t < T; ++t) {
+    const int f = fmt(t);
+    if (f != ARC_STEP_BF16 && f != ARC_STEP_NVFP4 && f != ARC_STEP_FP8) return ARC_ERR_INVALID_ARG;
+    if (f == ARC_STEP_FP8)
+      for (int i = 0; i < blk->n_sublayers; ++i) {
+        const arc_swiglu_sublayer& L = blk->sublayers[i];
+        if (!L.gateup_fp8 || !L.gateup_fp8_scale || !L.down_fp8 || !L.down_fp8_scale) return ARC_ERR_INVALID_ARG;
+      }
+  }
+  int sms = 0;
+  if (beta != 1.0f) {
+    const arc_status dc = device_check(&sms);
+    if (dc != ARC_OK) return dc;
+  }
   const size_t need = arc_recurrent_workspace_bytes(S_, blk);
   if (!workspace || ws_bytes < need) return ARC_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ARC_ERR_ALIGNMENT;
@@ -666,10 +795,10 @@ arc_status recurrent_run(void* h_bf16, int64_t S_, const arc_swiglu_block* blk, 
   const size_t qws_bytes = ws_bytes - off[6];
   arc_status st;
   for (int32_t t = 0; t < T; ++t) {
-    const bool low = low_step(t);
+    const int f = fmt(t);
     for (int i = 0; i < blk->n_sublayers; ++i) {
       const arc_swiglu_sublayer& L = blk->sublayers[i];
-      if (low) {
+      if (f == ARC_STEP_NVFP4) {
         if ((st = arc_quantize_act_nvfp4(h_bf16, S_, d, d, L.idx_gateup, L.r_gateup, L.rms_gain_bf16, blk->eps,
                                          nullptr, codes, sf, sA, qws, qws_bytes, stream)) != ARC_OK)
           return st;
@@ -680,14 +809,29 @@ arc_status recurrent_run(void* h_bf16, int64_t S_, const arc_swiglu_block* blk, 
         if ((st = arc_quantize_act_nvfp4(act, S_, F, F, L.idx_down, L.r_down, nullptr, 0.0f, nullptr, codes, sf,
                                          sA + 1, qws, qws_bytes, stream)) != ARC_OK)
           return st;
+        if (beta != 1.0f && (st = scale_bf16(h_bf16, S_, d, beta, stream, sms)) != ARC_OK) return st;
         if ((st = arc_gemm_nvfp4(codes, sf, sA + 1, L.down_codes, L.down_sf, L.down_scale, S_, d, F + L.r_down,
                                  h_bf16, d, h_bf16, d, stream)) != ARC_OK)
+          return st;
+      } else if (f == ARC_STEP_FP8) {
+        if ((st = arc_rmsnorm_bf16(h_bf16, S_, d, d, L.rms_gain_bf16, blk->eps, nrm, d, stream)) != ARC_OK) return st;
+        if ((st = arc_quantize_fp8(nrm, S_, d, d, nullptr, codes, d, sA, qws, qws_bytes, stream)) != ARC_OK) return st;
+        if ((st = arc_gemm_fp8(codes, d, sA, L.gateup_fp8, d, L.gateup_fp8_scale, S_, 2 * F, d, gu, 2 * F, nullptr, 0,
+                               stream)) != ARC_OK)
+          return st;
+        if ((st = arc_silu_mul_bf16(gu, S_, F, 2 * F, act, F, stream)) != ARC_OK) return st;
+        if ((st = arc_quantize_fp8(act, S_, F, F, nullptr, codes, F, sA + 1, qws, qws_bytes, stream)) != ARC_OK)
+          return st;
+        if (beta != 1.0f && (st = scale_bf16(h_bf16, S_, d, beta, stream, sms)) != ARC_OK) return st;
+        if ((st = arc_gemm_fp8(codes, F, sA + 1, L.down_fp8, F, L.down_fp8_scale, S_, d, F, h_bf16, d, h_bf16, d,
+                               stream)) != ARC_OK)
           return st;
       } else {
         if ((st = arc_rmsnorm_bf16(h_bf16, S_, d, d, L.rms_gain_bf16, blk->eps, nrm, d, stream)) != ARC_OK) return st;
         if ((st = arc_gemm_bf16(nrm, d, L.w_gateup_bf16, d, S_, 2 * F, d, gu, 2 * F, nullptr, 0, stream)) != ARC_OK)
           return st;
         if ((st = arc_silu_mul_bf16(gu, S_, F, 2 * F, act, F, stream)) != ARC_OK) return st;
+        if (beta != 1.0f && (st = scale_bf16(h_bf16, S_, d, beta, stream, sms)) != ARC_OK) return st;
         if ((st = arc_gemm_bf16(act, F, L.w_down_bf16, F, S_, d, F, h_bf16, d, h_bf16, d, stream)) != ARC_OK)
           return st;
       }
@@ -700,15 +844,16 @@ arc_status recurrent_run(void* h_bf16, int64_t S_, const arc_swiglu_block* blk, 
 arc_status arc_recurrent_prefill(void* h_bf16, int64_t S_, const arc_swiglu_block* blk, int32_t T, int32_t k_low,
                                  void* workspace, size_t ws_bytes, arc_stream_t stream) {
   if (k_low < 0) return ARC_ERR_INVALID_ARG;
-  return recurrent_run(h_bf16, S_, blk, T, [k_low](int32_t t) { return t < k_low; }, workspace, ws_bytes, stream);
+  return recurrent_run(h_bf16, S_, blk, T, [k_low](int32_t t) { return t < k_low ? ARC_STEP_NVFP4 : ARC_STEP_BF16; },
+                       workspace, ws_bytes, stream);
 }
 
 arc_status arc_recurrent_prefill_schedule(void* h_bf16, int64_t S_, const arc_swiglu_block* blk, int32_t T,
                                           const uint8_t* low_steps, void* workspace, size_t ws_bytes,
                                           arc_stream_t stream) {
   if (T > 0 && !low_steps) return ARC_ERR_INVALID_ARG;
-  return recurrent_run(h_bf16, S_, blk, T, [low_steps](int32_t t) { return low_steps[t] != 0; }, workspace,
-                       ws_bytes, stream);
+  return recurrent_run(h_bf16, S_, blk, T, [low_steps](int32_t t) { return static_cast<int>(low_steps[t]); },
+                       workspace, ws_bytes, stream);
 }
 
 arc_status arc_last_device_status(arc_stream_t stream) {

@@ -55,6 +55,14 @@ struct QuantArgs {
   uint64_t wait_ns;  // bound on the reordered kernel's waits (one that runs out sets the timeout status)
 };
 
+// Read-only 16-byte load that allocates in L1: two lanes' loads of one 32-byte sector then
+// fetch it from L2 once.
+__device__ __forceinline__ uint4 ld_nc_v4_l1(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -63,6 +71,17 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   return v;
 }
 
+
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t ldg_nc_u16(const void* p) {
+  uint16_t v;
+  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
 
 __device__ __forceinline__ bool in_safe_range(float v) {
   return v >= 8.077935669463161e-28f && v <= 1.2379400392853803e27f;  // [2^-90, 2^90]
@@ -324,239 +343,498 @@ __global__ void __launch_bounds__(256) k_amax(const __nv_bfloat16* __restrict__ 
   cta_max_to(max(mx & 0xFFFFu, mx >> 16) << 16, &partials[blockIdx.x]);
 }
 
-constexpr int kQRowThreads = 128;  // one CTA codes one row at a time
-constexpr int kQRowDepth = 2;      // 16-element blocks in flight per thread (4 measured 8% slower: register pressure)
+// ---------------------------------------------------------------------------------------------
+// The natural-order quantizer: one warp codes one whole row at a time; lane l codes blocks
+// 32 j + l of the row (two 32-block segments, 2 KB of the row, in flight per warp), so a row never
+// leaves its warp and the outlier channels of the row are handled with warp synchronisation only.
+// ---------------------------------------------------------------------------------------------
+
+constexpr int kQRowMaxWarps = 8;           // warps per CTA (fewer when the per-warp tables are large)
 constexpr int kQRowsSmemMax = 200 * 1024;  // largest dynamic shared memory the call accepts
 
-// Dynamic shared memory of k_quant_rows:
-//   idx_s     int32 [r]        the outlier channels (-1 for an out-of-range entry)
-//   blk_slot  int16 [K/16]     slot of each 16-channel block holding an outlier, else -1
-//   slots     [nslot]          48 bytes per outlier block of the current row: values, codes, d
-//   stash     float [r]        the row's residuals (values for weights) in idx order
+__host__ __device__ constexpr size_t qalign16(size_t x) { return (x + 15) / 16 * 16; }
 __host__ __device__ constexpr int qrows_nslot(int K, int r) { return r < K / 16 ? r : K / 16; }
-__host__ __device__ constexpr size_t qrows_smem_bytes(int K, int r) {
-  return (static_cast<size_t>(r) * 4 + 15) / 16 * 16 + (static_cast<size_t>(K / 16) * 2 + 15) / 16 * 16 +
-         static_cast<size_t>(qrows_nslot(K, r)) * 48 + (static_cast<size_t>(r) * 4 + 15) / 16 * 16 + 16;
+// Dynamic shared memory of k_quant_rows:
+//   shared by the CTA:  idx_s int32 [r] (the outlier channels, -1 for an out-of-range entry),
+//                       blk_slot int16 [K/16] (slot of each block holding an outlier, else -1)
+//   per warp:           slots uint4 [nslot] (the codes and d of the row's outlier blocks),
+//                       stash float [r] (the row's residuals, or values for weights, in idx order)
+__host__ __device__ constexpr size_t qrows_shared_bytes(int K, int r) {
+  return r > 0 ? qalign16(static_cast<size_t>(r) * 4) + qalign16(static_cast<size_t>(K / 16) * 2) : 0;
+}
+__host__ __device__ constexpr size_t qrows_warp_bytes(int K, int r) {
+  return static_cast<size_t>(qrows_nslot(K, r)) * 16 + qalign16(static_cast<size_t>(r) * 4);
+}
+// Warps per CTA that fit the shared-memory limit (0: the request is too large).
+__host__ __device__ constexpr int qrows_warps(int K, int r) {
+  return qrows_shared_bytes(K, r) + qrows_warp_bytes(K, r) > static_cast<size_t>(kQRowsSmemMax) ? 0
+         : qrows_warp_bytes(K, r) == 0 ? kQRowMaxWarps
+         : ((kQRowsSmemMax - qrows_shared_bytes(K, r)) / qrows_warp_bytes(K, r) < static_cast<size_t>(kQRowMaxWarps)
+                ? static_cast<int>((kQRowsSmemMax - qrows_shared_bytes(K, r)) / qrows_warp_bytes(K, r))
+                : kQRowMaxWarps);
+}
+__host__ __device__ constexpr size_t qrows_smem_bytes(int K, int r, int warps) {
+  return qrows_shared_bytes(K, r) + static_cast<size_t>(warps) * qrows_warp_bytes(K, r);
+}
+
+// max(|x|) of 16 bf16 values (8 packed pairs), as the fp32 value of the largest bf16 magnitude.
+// max.xorsign.abs keeps the larger magnitude of each half (its sign bit is not used).
+__device__ __forceinline__ uint32_t bf16x2_maxabs(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ float absmax16_bf16(const uint32_t (&w)[8]) {
+  const uint32_t m = bf16x2_maxabs(bf16x2_maxabs(bf16x2_maxabs(w[0], w[1]), bf16x2_maxabs(w[2], w[3])),
+                                   bf16x2_maxabs(bf16x2_maxabs(w[4], w[5]), bf16x2_maxabs(w[6], w[7])));
+  const uint32_t both = bf16x2_maxabs(m, __byte_perm(m, 0, 0x1032));  // both halves hold the maximum
+  return __uint_as_float(both & 0x7FFF0000u);
+}
+
+// Scale byte E4M3((amax / 6) / s) with both divides correctly rounded, for a tensor scale s in
+// [2^-80, 2^80] (rcp_s = RN(1/s), rcp6 = RN(1/6)). Exact by Markstein's correction wherever it
+// can change the byte: for amax below 2^-90 the quotient is below 2^-10 / 6 and the byte is 0
+// whatever its last bits; a quotient outside [2^-20, 2^20] gives 0 or 448 (infinity saturates).
+__device__ __forceinline__ uint32_t scale_byte_fast(float amax, float s, float rcp_s, float rcp6) {
+  const float t1 = div_rn_from_rcp(amax, 6.0f, rcp6);
+  const float q0 = __fmul_rn(t1, rcp_s);
+  const float qc = __fmaf_rn(__fmaf_rn(-q0, s, t1), rcp_s, q0);
+  return e4m3_rn_sat((q0 >= 9.5367431640625e-07f && q0 <= 1048576.0f) ? qc : q0);
+}
+
+// Codes of 16 values (8 fp32 pairs) against the decode scale of a table entry (d, -RN(1/d)) with
+// d in [2^-89, 2^89]: the negated correctly rounded quotients, E2M1 with the sign bits flipped
+// back (see encode16_nr); all zero when d == 0.
+__device__ __forceinline__ uint2 encode16_pairs(const uint64_t (&p)[8], float2 dn) {
+  const uint64_t nr2 = f2_pack(dn.y, dn.y), d2 = f2_pack(dn.x, dn.x);
+  float lo[8], hi[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    f2_unpack(neg_div2_rn(p[j], d2, nr2), lo[2 * j], lo[2 * j + 1]);
+    f2_unpack(neg_div2_rn(p[4 + j], d2, nr2), hi[2 * j], hi[2 * j + 1]);
+  }
+  const uint32_t a = e2m1x8_rn_sat(lo) ^ 0x88888888u, b = e2m1x8_rn_sat(hi) ^ 0x88888888u;
+  return dn.x != 0.0f ? make_uint2(a, b) : make_uint2(0u, 0u);
+}
+
+// One block of 16 fp32 values (any magnitudes) with the general scale and divide paths: used
+// when the tensor scale is outside [2^-80, 2^80], and for a saturated scale byte under a static
+// tensor scale (the quotients may then be too large for the reciprocal form).
+__device__ __forceinline__ void code_block_general(const float* v, float s, uint32_t* sfb_out, uint2* cc_out) {
+  float am = 0.0f;
+  for (int e = 0; e < 16; ++e) am = fmaxf(am, fabsf(v[e]));
+  const uint32_t sfb = e4m3_rn_sat(__fdiv_rn(__fdiv_rn(am, 6.0f), s));
+  const float d = __fmul_rn(e4m3_value(sfb), s);
+  uint2 cc = make_uint2(0u, 0u);
+  if (d != 0.0f) {
+    float lo[8], hi[8];
+    for (int e = 0; e < 8; ++e) {
+      lo[e] = __fdiv_rn(v[e], d);
+      hi[e] = __fdiv_rn(v[8 + e], d);
+    }
+    cc = make_uint2(e2m1x8_rn_sat(lo), e2m1x8_rn_sat(hi));
+  }
+  *sfb_out = sfb;
+  *cc_out = cc;
 }
 
 template <bool RMS>
-__global__ void __launch_bounds__(kQRowThreads, 6) k_quant_rows(QuantArgs a, int mpad) {
+__global__ void __launch_bounds__(kQRowMaxWarps * 32, 4) k_quant_rows(QuantArgs a, int mpad) {
   extern __shared__ __align__(16) uint8_t qsm[];
-  const int nblk = a.K >> 4;
-  const int tid = threadIdx.x, lane = tid & 31;
-  constexpr int NT = kQRowThreads;
+  const int nwarps = static_cast<int>(blockDim.x >> 5);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nblk = a.K >> 4, r = a.r;
+  const int nslot = qrows_nslot(a.K, r);
   int32_t* idx_s = reinterpret_cast<int32_t*>(qsm);
-  int16_t* blk_slot = reinterpret_cast<int16_t*>(qsm + (static_cast<size_t>(a.r) * 4 + 15) / 16 * 16);
-  uint4* slots = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(blk_slot) +
-                                          (static_cast<size_t>(nblk) * 2 + 15) / 16 * 16);  // 3 x 16 B each
-  float* stash = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(slots) +
-                                          static_cast<size_t>(qrows_nslot(a.K, a.r)) * 48);
-  __shared__ int nslot_sh;
-  // the first batch of a row's blocks is loaded while the previous row finishes its residual
-  // step, so each row starts with its data in flight; the first row's at entry, under the set-up
-  uint4 raw[kQRowDepth][2];
-  auto load_batch = [&](const __nv_bfloat16* rp, int b0) {
-#pragma unroll
-    for (int i = 0; i < kQRowDepth; ++i) {
-      const int b = b0 + NT * i + tid;
-      if (b < nblk) {
-        raw[i][0] = ld_nc_v4(rp + 16 * b);
-        raw[i][1] = ld_nc_v4(rp + 16 * b + 8);
-      } else {
-        raw[i][0] = raw[i][1] = make_uint4(0, 0, 0, 0);
-      }
+  int16_t* blk_slot = reinterpret_cast<int16_t*>(qsm + qalign16(static_cast<size_t>(r) * 4));
+  uint8_t* wsm = qsm + qrows_shared_bytes(a.K, r) + static_cast<size_t>(warp) * qrows_warp_bytes(a.K, r);
+  uint4* slots = reinterpret_cast<uint4*>(wsm);
+  float* stash = reinterpret_cast<float*>(wsm + static_cast<size_t>(nslot) * 16);
+
+  // ---- outlier tables (before the wait: they overlap the first kernel); out-of-range entries
+  // are reported and left out
+  if (r > 0) {
+    __shared__ int nslot_sh;
+    for (int b = tid; b < nblk; b += blockDim.x) blk_slot[b] = -1;
+    if (tid == 0) nslot_sh = 0;
+    __syncthreads();
+    for (int j = tid; j < r; j += blockDim.x) {
+      const int c = a.idx[j];
+      const bool ok = static_cast<unsigned>(c) < static_cast<unsigned>(a.K);
+      if (!ok && blockIdx.x == 0) set_status(kStatusInvalidArg);
+      idx_s[j] = ok ? c : -1;
+      if (ok) blk_slot[c >> 4] = -2;
     }
-  };
-  if (static_cast<int>(blockIdx.x) < a.M) load_batch(a.x + static_cast<int64_t>(blockIdx.x) * a.ldx, 0);
-
-  // outlier tables (before the wait: they overlap the first kernel); out-of-range entries are
-  // reported and left out
-  for (int b = tid; b < nblk; b += NT) blk_slot[b] = -1;
-  if (tid == 0) nslot_sh = 0;
-  __syncthreads();
-  for (int j = tid; j < a.r; j += NT) {
-    const int c = a.idx[j];
-    const bool ok = static_cast<unsigned>(c) < static_cast<unsigned>(a.K);
-    if (!ok && blockIdx.x == 0) set_status(kStatusInvalidArg);
-    idx_s[j] = ok ? c : -1;
-    if (ok) blk_slot[c >> 4] = -2;
+    __syncthreads();
+    for (int b = tid; b < nblk; b += blockDim.x)
+      if (blk_slot[b] == -2) blk_slot[b] = static_cast<int16_t>(atomicAdd(&nslot_sh, 1));
   }
-  __syncthreads();
-  for (int b = tid; b < nblk; b += NT)
-    if (blk_slot[b] == -2) blk_slot[b] = static_cast<int16_t>(atomicAdd(&nslot_sh, 1));
 
-  // ---- tensor scale
+  // ---- tensor scale and the decode-scale table
   pdl_wait();
   float s;
   {
     __shared__ float s_sh;
-    s = a.static_scale ? *a.static_scale : cta_tensor_scale(a);
+    s = cta_tensor_scale(a);
     if (tid == 0) s_sh = s;
     __syncthreads();
     s = s_sh;
   }
   if (blockIdx.x == 0 && tid == 0) *a.scale_out = s;
   const float rcp_s = __frcp_rn(s), rcp6 = __frcp_rn(6.0f);
-  // decode scale d = E4M3value(byte) * s and -RN(1/d) for every scale byte (0..126)
-  __shared__ float2 dtab[128];
-  for (int i = tid; i < 128; i += NT) {
+  // with s in [2^-80, 2^80] every nonzero decode scale lies in [2^-89, 2^89], where the
+  // reciprocal forms are exact; otherwise every block takes the general path
+  const bool fast = s >= 8.271806125530277e-25f && s <= 1.2089258196146292e24f;
+  // a static scale may be too small for the data: a block whose byte saturates then takes the
+  // general path (with the dynamic scale no quotient exceeds 2688 / 2^-9)
+  const bool check_sat = a.static_scale != nullptr;
+  __shared__ float2 dtab[128];  // decode scale d and -RN(1/d) of scale byte i (entry 0: d = 0)
+  for (int i = tid; i < 128; i += blockDim.x) {
     const float dd = __fmul_rn(e4m3_value(static_cast<uint32_t>(i)), s);
-    dtab[i] = make_float2(dd, in_safe_range(dd) ? -__frcp_rn(dd) : 0.0f);
+    dtab[i] = make_float2(dd, (fast && i > 0) ? -__frcp_rn(dd) : 0.0f);
   }
   __syncthreads();
-  const int64_t cpitch = a.kpad >> 1;
-  const int nres = a.r >> 4, ntail = (a.kpad - a.K) >> 4;
 
-  for (int m = blockIdx.x; m < mpad; m += gridDim.x) {
-    if (m >= a.M) {  // rows padding the scale layout to a multiple of 128 carry zero scales
-      for (int kb = tid; kb < (a.kpad >> 4); kb += NT) a.sf[sf_offset(m, kb, a.katoms)] = 0;
-      continue;
+  const int64_t cpitch = a.kpad >> 1;
+  const int nseg = (nblk + 31) >> 5;
+  const int nres = r >> 4, ntail = (a.kpad - a.K) >> 4;
+  const bool keep_slots = r > 0 && !a.dup;  // activations need the codes and d of outlier blocks
+
+  // Rows of this warp: m = blockIdx.x + gridDim.x * j for j = warp, warp + nwarps, ... The row's
+  // 32-block segments are double-buffered in registers: segment s + 1 (or the next row's first
+  // segment) is loaded while segment s is coded.
+  const __nv_bfloat16* __restrict__ xg = a.x;
+  auto row_of = [&](int64_t jj) { return static_cast<int64_t>(blockIdx.x) + static_cast<int64_t>(gridDim.x) * jj; };
+  auto load_seg = [&](int64_t m, int seg, uint4& lo, uint4& hi) {
+    const int b = seg * 32 + lane;
+    lo = hi = make_uint4(0, 0, 0, 0);
+    if (m < a.M && b < nblk) {
+      const __nv_bfloat16* p = xg + m * a.ldx + 16 * b;
+      lo = ld_nc_v4_l1(p);
+      hi = ld_nc_v4_l1(p + 8);
     }
-    const __nv_bfloat16* row = a.x + static_cast<int64_t>(m) * a.ldx;
-    uint8_t* crow = a.codes + static_cast<int64_t>(m) * cpitch;
+  };
+  int64_t jrow = warp;
+  int64_t m = row_of(jrow);
+  uint4 cur_lo, cur_hi;
+  load_seg(m, 0, cur_lo, cur_hi);
+  for (; m < mpad; m = row_of(jrow += nwarps)) {
     // scale byte of (m, kb) at sf_row + (kb / 4) * 512 + kb % 4
-    uint8_t* sf_row = a.sf + static_cast<int64_t>(m >> 7) * a.katoms * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4;
+    uint8_t* sf_row = a.sf + (m >> 7) * a.katoms * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4;
+    if (m >= a.M) {  // rows padding the scale layout to a multiple of 128 carry zero scales
+      for (int kb = lane; kb < (a.kpad >> 4); kb += 32) sf_row[(kb >> 2) * 512 + (kb & 3)] = 0;
+      continue;  // every later row of the warp pads too: nothing to prefetch
+    }
+    const __nv_bfloat16* row = xg + m * a.ldx;
+    uint8_t* crow = a.codes + m * cpitch;
     double inv = 0.0;
     if (RMS) inv = a.inv_rms[m];
-    // ---- primary blocks: thread t codes blocks b0 + 128 i + t
-    for (int b0 = 0; b0 < nblk; b0 += NT * kQRowDepth) {
-      if (b0 > 0) load_batch(row, b0);
+    // ---- primary blocks
+    for (int seg = 0; seg < nseg; ++seg) {
+      uint4 nxt_lo, nxt_hi;
+      if (seg + 1 < nseg)
+        load_seg(m, seg + 1, nxt_lo, nxt_hi);
+      else
+        load_seg(row_of(jrow + nwarps), 0, nxt_lo, nxt_hi);  // the warp's next row
+      const int b = seg * 32 + lane;
+      const bool valid = b < nblk;
+      uint32_t w[8] = {cur_lo.x, cur_lo.y, cur_lo.z, cur_lo.w, cur_hi.x, cur_hi.y, cur_hi.z, cur_hi.w};
+      if (RMS && valid) {
+        // RMSNorm prologue: each value becomes bf16((h * inv) * g), repacked as bf16 pairs
+        const uint4 g0 = ld_nc_v4_l1(a.gain + 16 * b), g1 = ld_nc_v4_l1(a.gain + 16 * b + 8);
+        const uint32_t g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
-      for (int i = 0; i < kQRowDepth; ++i) {
-        const int b = b0 + NT * i + tid;
-        if (b0 + NT * i >= nblk) break;  // uniform: no block of this batch position exists
-        const bool valid = b < nblk;
-        const uint32_t w[8] = {raw[i][0].x, raw[i][0].y, raw[i][0].z, raw[i][0].w,
-                               raw[i][1].x, raw[i][1].y, raw[i][1].z, raw[i][1].w};
+        for (int e = 0; e < 8; ++e)
+          w[e] = pack_bf16x2_rn(rms_apply(bf16_lo(w[e]), inv, bf16_lo(g[e])), rms_apply(bf16_hi(w[e]), inv, bf16_hi(g[e])));
+      }
+      uint64_t p[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) p[e] = f2_pack(bf16_lo(w[e]), bf16_hi(w[e]));
+      uint32_t sfb;
+      uint2 cc;
+      if (fast) {
+        sfb = scale_byte_fast(absmax16_bf16(w), s, rcp_s, rcp6);
+        cc = encode16_pairs(p, dtab[sfb]);
+        if (check_sat && sfb == 0x7Eu) {
+          float v[16];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f2_unpack(p[e], v[2 * e], v[2 * e + 1]);
+          code_block_general(v, s, &sfb, &cc);
+        }
+      } else {
         float v[16];
-        float amax;
-        if (RMS) {
-          uint4 g0 = make_uint4(0, 0, 0, 0), g1 = g0;
-          if (valid) {
-            g0 = ld_nc_v4(a.gain + 16 * b);
-            g1 = ld_nc_v4(a.gain + 16 * b + 8);
-          }
-          const uint32_t gs[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            v[2 * j] = rms_apply(bf16_lo(w[j]), inv, bf16_lo(gs[j]));
-            v[2 * j + 1] = rms_apply(bf16_hi(w[j]), inv, bf16_hi(gs[j]));
-          }
-          const float a0 = fmax3_abs(v[0], v[1], v[2]), a1 = fmax3_abs(v[3], v[4], v[5]),
-                      a2 = fmax3_abs(v[6], v[7], v[8]), a3 = fmax3_abs(v[9], v[10], v[11]),
-                      a4 = fmax3_abs(v[12], v[13], v[14]);
-          amax = fmaxf(fmax3(a0, a1, a2), fmax3(a3, a4, fabsf(v[15])));
-        } else {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            v[2 * j] = bf16_lo(w[j]);
-            v[2 * j + 1] = bf16_hi(w[j]);
-          }
-          // |bf16| orders like its bit pattern: the block maximum on packed halves
-          const uint32_t m01 = __vmaxu2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu);
-          const uint32_t m23 = __vmaxu2(w[2] & 0x7FFF7FFFu, w[3] & 0x7FFF7FFFu);
-          const uint32_t m45 = __vmaxu2(w[4] & 0x7FFF7FFFu, w[5] & 0x7FFF7FFFu);
-          const uint32_t m67 = __vmaxu2(w[6] & 0x7FFF7FFFu, w[7] & 0x7FFF7FFFu);
-          const uint32_t mw = __vmaxu2(__vmaxu2(m01, m23), __vmaxu2(m45, m67));
-          amax = __uint_as_float(max(mw & 0xFFFFu, mw >> 16) << 16);
-        }
-        const uint32_t sfv = block_sf(amax, s, rcp_s, rcp6);
-        const float2 dn = dtab[sfv];
-        const float d = dn.x;
-        uint2 cc = make_uint2(0u, 0u);
-        if (d != 0.0f) {
-          uint64_t p[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) p[j] = f2_pack(v[2 * j], v[2 * j + 1]);
-          cc = encode16_nr(p, d, dn.y);
-        }
-        if (valid) *reinterpret_cast<uint2*>(crow + 8 * b) = cc;
-        // a block holding outlier channels keeps its values (bf16: the RMSNorm output is
-        // bf16-rounded), codes and d for the residual step below
-        const int sl = (valid && a.r > 0) ? blk_slot[b] : -1;
-        if (sl >= 0) {
-          uint4* dst = slots + 3 * sl;
-          if (RMS) {
-            dst[0] = make_uint4(pack_bf16x2_rn(v[0], v[1]), pack_bf16x2_rn(v[2], v[3]), pack_bf16x2_rn(v[4], v[5]),
-                                pack_bf16x2_rn(v[6], v[7]));
-            dst[1] = make_uint4(pack_bf16x2_rn(v[8], v[9]), pack_bf16x2_rn(v[10], v[11]),
-                                pack_bf16x2_rn(v[12], v[13]), pack_bf16x2_rn(v[14], v[15]));
-          } else {
-            dst[0] = raw[i][0];
-            dst[1] = raw[i][1];
-          }
-          dst[2] = make_uint4(cc.x, cc.y, __float_as_uint(d), 0u);
-        }
-        // scale bytes: lanes 4i..4i+3 hold blocks b..b+3 (b % 4 == 0 at lane 4i), which sit in
-        // four consecutive bytes of the swizzled layout
-        const uint32_t my = valid ? sfv : 0u;
-        const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, my, 1), s2 = __shfl_down_sync(0xFFFFFFFFu, my, 2),
-                       s3 = __shfl_down_sync(0xFFFFFFFFu, my, 3);
-        if (valid && (lane & 3) == 0) {
-          uint8_t* dst = sf_row + (b >> 2) * 512;
-          if (b + 3 < nblk) {
-            *reinterpret_cast<uint32_t*>(dst) = my | (s1 << 8) | (s2 << 16) | (s3 << 24);
-          } else {
-            dst[0] = static_cast<uint8_t>(my);
-            if (b + 1 < nblk) dst[1] = static_cast<uint8_t>(s1);
-            if (b + 2 < nblk) dst[2] = static_cast<uint8_t>(s2);
-          }
+        for (int e = 0; e < 8; ++e) f2_unpack(p[e], v[2 * e], v[2 * e + 1]);
+        code_block_general(v, s, &sfb, &cc);
+      }
+      if (valid) {
+        *reinterpret_cast<uint2*>(crow + 8 * b) = cc;
+        sf_row[(b >> 2) * 512 + (b & 3)] = static_cast<uint8_t>(sfb);
+        if (keep_slots) {
+          const int sl = blk_slot[b];
+          if (sl >= 0) slots[sl] = make_uint4(cc.x, cc.y, __float_as_uint(dtab[sfb].x), 0u);
         }
       }
+      cur_lo = nxt_lo;
+      cur_hi = nxt_hi;
     }
-    {
-      const int mn = m + static_cast<int>(gridDim.x);
-      if (mn < a.M) load_batch(a.x + static_cast<int64_t>(mn) * a.ldx, 0);
-    }
-    if (a.r > 0) {
+    if (r > 0) {
       // ---- outlier channels: residual x - E2M1(code) * d (activations) or the value itself
-      // (weights), from the kept blocks
-      __syncthreads();
-      for (int j = tid; j < a.r; j += NT) {
-        const int c = idx_s[j];
+      // (weights); with the prologue, x is normalised again exactly as the primary pass did
+      __syncwarp();
+      auto residual = [&](int jj, int c, uint32_t hb) {
         float res = 0.0f;
         if (c >= 0) {
-          const uint4* src = slots + 3 * blk_slot[c >> 4];
-          const int e = c & 15;
-          const uint4 vw = src[e >> 3];
-          const int wi = (e >> 1) & 3;
-          const uint32_t word = wi == 0 ? vw.x : wi == 1 ? vw.y : wi == 2 ? vw.z : vw.w;
-          const float xv = (e & 1) ? bf16_hi(word) : bf16_lo(word);
+          float xv = __uint_as_float(hb << 16);
+          if (RMS) xv = rms_apply(xv, inv, __uint_as_float(ldg_nc_u16(a.gain + c) << 16));
           res = xv;
           if (!a.dup) {
-            const uint4 meta = src[2];
+            const uint4 meta = slots[blk_slot[c >> 4]];
+            const int e = c & 15;
             const uint32_t code = (((e < 8) ? meta.x : meta.y) >> (4 * (e & 7))) & 15u;
             res = __fsub_rn(xv, __fmul_rn(e2m1_value(code), __uint_as_float(meta.z)));
           }
         }
-        stash[j] = res;
+        stash[jj] = res;
+      };
+      for (int jj = lane; jj < r; jj += 32) {
+        const int c = idx_s[jj];
+        residual(jj, c, c >= 0 ? ldg_nc_u16(row + c) : 0u);
       }
-      __syncthreads();
+      __syncwarp();
     }
     // ---- appended residual blocks (in idx order, same tensor scale) and zero padding to K_pad
-    for (int rb = tid; rb < ntail; rb += NT) {
-      uint32_t sfv = 0u;
+    for (int rb = lane; rb < ntail; rb += 32) {
+      uint32_t sfb = 0u;
       uint2 cc = make_uint2(0u, 0u);
       if (rb < nres) {
         float v[16];
+        const float4* src = reinterpret_cast<const float4*>(stash + 16 * rb);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] = stash[16 * rb + e];
-        const float a0 = fmax3_abs(v[0], v[1], v[2]), a1 = fmax3_abs(v[3], v[4], v[5]),
-                    a2 = fmax3_abs(v[6], v[7], v[8]), a3 = fmax3_abs(v[9], v[10], v[11]),
-                    a4 = fmax3_abs(v[12], v[13], v[14]);
-        sfv = block_sf(fmaxf(fmax3(a0, a1, a2), fmax3(a3, a4, fabsf(v[15]))), s, rcp_s, rcp6);
-        const float2 dn = dtab[sfv];
-        if (dn.x != 0.0f) {
+        for (int q = 0; q < 4; ++q) {
+          const float4 f = src[q];
+          v[4 * q] = f.x, v[4 * q + 1] = f.y, v[4 * q + 2] = f.z, v[4 * q + 3] = f.w;
+        }
+        if (fast) {
+          const float a0 = fmax3_abs(v[0], v[1], v[2]), a1 = fmax3_abs(v[3], v[4], v[5]),
+                      a2 = fmax3_abs(v[6], v[7], v[8]), a3 = fmax3_abs(v[9], v[10], v[11]),
+                      a4 = fmax3_abs(v[12], v[13], v[14]);
+          sfb = scale_byte_fast(fmaxf(fmax3(a0, a1, a2), fmax3(a3, a4, fabsf(v[15]))), s, rcp_s, rcp6);
           uint64_t p[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) p[j] = f2_pack(v[2 * j], v[2 * j + 1]);
-          cc = encode16_nr(p, dn.x, dn.y);
+          for (int e = 0; e < 8; ++e) p[e] = f2_pack(v[2 * e], v[2 * e + 1]);
+          cc = encode16_pairs(p, dtab[sfb]);
+          if (check_sat && sfb == 0x7Eu) code_block_general(v, s, &sfb, &cc);
+        } else {
+          code_block_general(v, s, &sfb, &cc);
         }
       }
       *reinterpret_cast<uint2*>(crow + ((a.K + 16 * rb) >> 1)) = cc;
       const int kb = nblk + rb;
-      sf_row[(kb >> 2) * 512 + (kb & 3)] = static_cast<uint8_t>(sfv);
+      sf_row[(kb >> 2) * 512 + (kb & 3)] = static_cast<uint8_t>(sfb);
     }
+    __syncwarp();  // the warp's slots and stash are reused by its next row
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// MXFP4 with augmented residual channels (ARCQuant, Resultaten / Generaliseerbaarheid: the
+// approach extends to MXFP4), read as the OCP microscaling format: 32 consecutive values share
+// one power-of-two scale X = 2^(floor(log2 amax) - 2), stored as the E8M0 byte
+// max(exponent field of amax - 2, 0); elements are E2M1 of x / X with the sign of x (an all-zero
+// block has byte 0 and zero codes); no tensor scale. The residual of outlier channel c is
+// x_c - E2M1(code_c) * X (exact product, fp32 subtract); the residuals in idx order form r/32
+// blocks coded the same way after the K primary channels; weights append the channel itself.
+// x / X is the single correctly rounded product x * 2^(127 - byte), so no division is needed and
+// there is no tensor-wide pass: the quantizer is one kernel that reads X once.
+//
+// Layout: codes [rows, K_pad/2] as for NVFP4; scale bytes in 512-byte atoms of 128 rows x 4
+// scales (128 K-elements), atom (i, j) at (i * ceil(K_pad/128) + j) * 512, row m / scale column
+// kb inside at (m%32)*16 + ((m/32)%4)*4 + kb%4 (pad columns and pad rows zero).
+//
+// Work split: one warp per row at a time, as k_quant_rows; lanes 2i and 2i+1 code the two halves
+// of block i of a 16-block segment (each lane 16 values, one 32-byte sector), the block maximum
+// joined by one shuffle.
+// ---------------------------------------------------------------------------------------------
+
+constexpr int kQMxMaxWarps = 8;
+constexpr uint32_t kMxZeroBlock = 0xFFu;  // per-warp scale table: block whose maximum is zero
+
+// Dynamic shared memory of k_quant_mx_rows: idx_s int32 [r] (shared), then per warp the row's
+// scale bytes uint8 [K/32] (0xFF for an all-zero block) and stash float [r].
+__host__ __device__ constexpr size_t qmx_shared_bytes(int r) { return qalign16(static_cast<size_t>(r) * 4); }
+__host__ __device__ constexpr size_t qmx_warp_bytes(int K, int r) {
+  return r > 0 ? qalign16(static_cast<size_t>(K / 32)) + qalign16(static_cast<size_t>(r) * 4) : 0;
+}
+__host__ __device__ constexpr int qmx_warps(int K, int r) {
+  return qmx_shared_bytes(r) + qmx_warp_bytes(K, r) > static_cast<size_t>(kQRowsSmemMax) ? 0
+         : qmx_warp_bytes(K, r) == 0 ? kQMxMaxWarps
+         : ((kQRowsSmemMax - qmx_shared_bytes(r)) / qmx_warp_bytes(K, r) < static_cast<size_t>(kQMxMaxWarps)
+                ? static_cast<int>((kQRowsSmemMax - qmx_shared_bytes(r)) / qmx_warp_bytes(K, r))
+                : kQMxMaxWarps);
+}
+__host__ __device__ constexpr size_t qmx_smem_bytes(int K, int r, int warps) {
+  return qmx_shared_bytes(r) + static_cast<size_t>(warps) * qmx_warp_bytes(K, r);
+}
+
+// E8M0 byte of a block maximum (fp32 bits): floor(log2 amax) - 2 + 127 clamped to [0, 254]; a
+// zero or subnormal maximum gives 0.
+__device__ __forceinline__ uint32_t mx_scale_byte(uint32_t amax_bits) {
+  return static_cast<uint32_t>(max(static_cast<int>((amax_bits >> 23) & 0xFFu) - 2, 0));
+}
+// 2^(127 - byte) (normal for every byte <= 252) and X = 2^(byte - 127) (subnormal for byte 0).
+__device__ __forceinline__ float mx_inv_scale(uint32_t sb) { return __uint_as_float((254u - sb) << 23); }
+__device__ __forceinline__ float mx_scale(uint32_t sb) { return sb ? __uint_as_float(sb << 23) : __uint_as_float(0x00400000u); }
+
+// Codes of 16 values (8 fp32 pairs) times 2^(127 - byte).
+__device__ __forceinline__ uint2 mx_encode16(const uint64_t (&p)[8], float inv) {
+  const uint64_t m2 = f2_pack(inv, inv);
+  float lo[8], hi[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    f2_unpack(f2_mul(p[j], m2), lo[2 * j], lo[2 * j + 1]);
+    f2_unpack(f2_mul(p[4 + j], m2), hi[2 * j], hi[2 * j + 1]);
+  }
+  return make_uint2(e2m1x8_rn_sat(lo), e2m1x8_rn_sat(hi));
+}
+
+struct QuantMxArgs {
+  const __nv_bfloat16* x;
+  int64_t ldx;
+  int M, K, r, kpad, katoms;  // katoms = ceil(K_pad / 128)
+  const int32_t* idx;
+  uint8_t* codes;
+  uint8_t* sf;
+  int dup;
+};
+
+__global__ void __launch_bounds__(kQMxMaxWarps * 32, 4) k_quant_mx_rows(QuantMxArgs a, int mpad) {
+  extern __shared__ __align__(16) uint8_t qsm[];
+  const int nwarps = static_cast<int>(blockDim.x >> 5);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nblk = a.K >> 5, r = a.r;
+  int32_t* idx_s = reinterpret_cast<int32_t*>(qsm);
+  uint8_t* wsm = qsm + qmx_shared_bytes(r) + static_cast<size_t>(warp) * qmx_warp_bytes(a.K, r);
+  uint8_t* sbrow = wsm;
+  float* stash = reinterpret_cast<float*>(wsm + qalign16(static_cast<size_t>(nblk)));
+  for (int j = tid; j < r; j += blockDim.x) {
+    const int c = a.idx[j];
+    const bool ok = static_cast<unsigned>(c) < static_cast<unsigned>(a.K);
+    if (!ok && blockIdx.x == 0) set_status(kStatusInvalidArg);
+    idx_s[j] = ok ? c : -1;
+  }
+  __syncthreads();
+
+  const int64_t cpitch = a.kpad >> 1;
+  const int nseg = (nblk + 15) >> 4;  // 16 blocks (512 values) per segment
+  const int nres = r >> 5;
+  const int ncols = 4 * a.katoms;     // scale columns including the atom padding
+  const int half = lane & 1;
+  auto row_of = [&](int64_t jj) { return static_cast<int64_t>(blockIdx.x) + static_cast<int64_t>(gridDim.x) * jj; };
+  auto load_seg = [&](int64_t m, int seg, uint4& lo, uint4& hi) {
+    const int b = seg * 16 + (lane >> 1);
+    lo = hi = make_uint4(0, 0, 0, 0);
+    if (m < a.M && b < nblk) {
+      const __nv_bfloat16* p = a.x + m * a.ldx + 32 * b + 16 * half;
+      lo = ld_nc_v4_l1(p);
+      hi = ld_nc_v4_l1(p + 8);
+    }
+  };
+  int64_t jrow = warp;
+  int64_t m = row_of(jrow);
+  uint4 cur_lo, cur_hi;
+  load_seg(m, 0, cur_lo, cur_hi);
+  for (; m < mpad; m = row_of(jrow += nwarps)) {
+    uint8_t* sf_row = a.sf + (m >> 7) * a.katoms * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4;
+    if (m >= a.M) {
+      for (int kb = lane; kb < ncols; kb += 32) sf_row[(kb >> 2) * 512 + (kb & 3)] = 0;
+      continue;
+    }
+    const __nv_bfloat16* row = a.x + m * a.ldx;
+    uint8_t* crow = a.codes + m * cpitch;
+    for (int seg = 0; seg < nseg; ++seg) {
+      uint4 nxt_lo, nxt_hi;
+      if (seg + 1 < nseg)
+        load_seg(m, seg + 1, nxt_lo, nxt_hi);
+      else
+        load_seg(row_of(jrow + nwarps), 0, nxt_lo, nxt_hi);
+      const int b = seg * 16 + (lane >> 1);
+      const uint32_t w[8] = {cur_lo.x, cur_lo.y, cur_lo.z, cur_lo.w, cur_hi.x, cur_hi.y, cur_hi.z, cur_hi.w};
+      const uint32_t mine = __float_as_uint(absmax16_bf16(w));
+      const uint32_t am = max(mine, __shfl_xor_sync(0xFFFFFFFFu, mine, 1));  // non-negative: bits order as values
+      const uint32_t sb = mx_scale_byte(am);
+      uint64_t p[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) p[e] = f2_pack(bf16_lo(w[e]), bf16_hi(w[e]));
+      uint2 cc = mx_encode16(p, mx_inv_scale(sb));
+      if (am == 0u) cc = make_uint2(0u, 0u);
+      if (b < nblk) {
+        *reinterpret_cast<uint2*>(crow + 16 * b + 8 * half) = cc;
+        if (!half) {
+          sf_row[(b >> 2) * 512 + (b & 3)] = static_cast<uint8_t>(sb);
+          if (r > 0) sbrow[b] = static_cast<uint8_t>(am == 0u ? kMxZeroBlock : sb);
+        }
+      }
+      cur_lo = nxt_lo;
+      cur_hi = nxt_hi;
+    }
+    if (r > 0) {
+      // ---- outlier channels: x - E2M1(code) * X (activations; the code recomputed from x and
+      // the block's byte, as the primary pass formed it) or x itself (weights)
+      __syncwarp();
+      for (int jj = lane; jj < r; jj += 32) {
+        const int c = idx_s[jj];
+        float res = 0.0f;
+        if (c >= 0) {
+          const float xv = __uint_as_float(ldg_nc_u16(row + c) << 16);
+          res = xv;
+          if (!a.dup) {
+            const uint32_t t = sbrow[c >> 5];
+            uint32_t code = 0u;
+            float X = mx_scale(0u);
+            if (t != kMxZeroBlock) {
+              float q[8] = {__fmul_rn(xv, mx_inv_scale(t)), 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+              code = e2m1x8_rn_sat(q) & 15u;
+              X = mx_scale(t);
+            }
+            res = __fsub_rn(xv, __fmul_rn(e2m1_value(code), X));
+          }
+        }
+        stash[jj] = res;
+      }
+      __syncwarp();
+    }
+    // ---- appended residual blocks (lane pairs, as the primary blocks) and zero padding
+    const int ntail = ncols - nblk;  // scale columns after the primary ones (residual blocks, padding)
+    for (int t0 = 0; t0 < ntail; t0 += 16) {
+      const int rb = t0 + (lane >> 1);
+      uint32_t am = 0u;
+      uint64_t p[8];
+      if (rb < nres) {
+        const float4* src = reinterpret_cast<const float4*>(stash + 32 * rb + 16 * half);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 f = src[q];
+          p[2 * q] = f2_pack(f.x, f.y);
+          p[2 * q + 1] = f2_pack(f.z, f.w);
+          am = max(am, max(max(__float_as_uint(fabsf(f.x)), __float_as_uint(fabsf(f.y))),
+                           max(__float_as_uint(fabsf(f.z)), __float_as_uint(fabsf(f.w)))));
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) p[e] = 0ull;
+      }
+      am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
+      const uint32_t sb = mx_scale_byte(am);
+      uint2 cc = mx_encode16(p, mx_inv_scale(sb));
+      if (am == 0u) cc = make_uint2(0u, 0u);
+      const int kb = nblk + rb;
+      if (rb < ntail) {
+        if (16 * kb + 8 * half < cpitch) *reinterpret_cast<uint2*>(crow + 16 * kb + 8 * half) = cc;
+        if (!half) sf_row[(kb >> 2) * 512 + (kb & 3)] = static_cast<uint8_t>(sb);
+      }
+    }
+    __syncwarp();
   }
 }
 
@@ -576,16 +854,6 @@ constexpr int kQReoSmemMax = 200 * 1024;  // two row buffers: K <= 51200 channel
 __host__ __device__ constexpr size_t qreo_row_bytes(int K) { return (static_cast<size_t>(K) * 2 + 127) / 128 * 128; }
 __host__ __device__ constexpr size_t qreo_smem_bytes(int K) { return 2 * qreo_row_bytes(K); }
 
-__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
-  uint16_t v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ uint32_t ldg_nc_u16(const void* p) {
-  uint16_t v;
-  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
-  return v;
-}
 
 // One CTA codes one row at a time; rows arrive by 1-D bulk copies into two shared-memory
 // buffers (the next row loads while this one is coded). Thread t codes primary blocks t, t + 256,

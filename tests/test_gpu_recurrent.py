@@ -46,7 +46,14 @@ def silu_within_one_ulp(got_bits, gu_bits):
     assert np.all(np.abs(got - want) <= ulp + 1e-38)
 
 
-def nvfp4_sublayer_teacher_forced(h, L, r):
+def sample_rows(S, n=8, seed=0):
+    """First and last rows plus n seeded random rows in between."""
+    rng = np.random.default_rng(seed)
+    mid = rng.choice(np.arange(4, S - 4), size=min(n, max(0, S - 8)), replace=False) if S > 8 else []
+    return np.unique(np.r_[0:min(4, S), max(0, S - 4):S, np.asarray(mid, dtype=np.int64)])
+
+
+def nvfp4_sublayer_teacher_forced(h, L, r, rows=None):
     S, d = h.shape
     hb = to_bits(h)
     g_bits = to_bits(L["gain"])
@@ -66,7 +73,7 @@ def nvfp4_sublayer_teacher_forced(h, L, r):
     wgu_bits = to_bits(L["wgu"])
     sw = O.tensor_scale(O.amax(wgu_bits))
     bc, bsf = O.pack_weight(wgu_bits, idx_gu, sw)
-    rows = np.r_[0:4, S - 4:S]
+    rows = sample_rows(S) if rows is None else rows
     ref = O.gemm_nvfp4_f64_matmul(c_ref, sf_ref, s_ref, bc, bsf, sw, rows=rows)
     gu_bits = to_bits(gu)
     assert normalized_gemm_error(gu_bits[rows], ref, row_norms(n_ref[rows]), row_norms(wgu_bits)) <= GEMM_TOL
@@ -93,7 +100,7 @@ def nvfp4_sublayer_teacher_forced(h, L, r):
     return h_new
 
 
-def bf16_sublayer_teacher_forced(h, L):
+def bf16_sublayer_teacher_forced(h, L, rows=None):
     S, d = h.shape
     hb = to_bits(h)
     g_bits = to_bits(L["gain"])
@@ -101,7 +108,7 @@ def bf16_sublayer_teacher_forced(h, L):
     n_bits = to_bits(n)
     np.testing.assert_array_equal(n_bits, O.rmsnorm(hb, g_bits, float(np.float32(EPS))))
     gu = arc.gemm_bf16(n, L["wgu"])
-    rows = np.r_[0:4, S - 4:S]
+    rows = sample_rows(S) if rows is None else rows
     wgu_bits = to_bits(L["wgu"])
     ref = O.gemm_bf16_f64(n_bits, wgu_bits, rows=rows)
     gu_bits = to_bits(gu)
@@ -181,3 +188,194 @@ def test_schedule_driver_equals_composed_steps(schedule):
     b = arc.recurrent_prefill(h0.clone(), blk, 4, k)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+@pytest.mark.slow
+def test_sublayers_teacher_forced_at_the_recurrent_workload_size():
+    # the recurrent workload's own shape: S = 4096 tokens, d = 2048, ffn = 8192, r = 64. At this
+    # size the fused RMSNorm quantizer codes many rows per CTA (its row loop and next-row
+    # prefetch), which the narrower tests never reach. Codes, scale bytes and tensor scales are
+    # compared over whole tensors, GEMM outputs on 64 seeded rows plus the first and last four.
+    c = W.RECURRENT
+    rec, h, subs = make_block(S=c["S"], d=c["d"], ffn=c["ffn"], r=c["r"])
+    rows = sample_rows(c["S"], n=64, seed=1)
+    h1 = nvfp4_sublayer_teacher_forced(h, subs[0], c["r"], rows=rows)
+    h2 = bf16_sublayer_teacher_forced(h1, subs[1], rows=rows)
+    assert torch.isfinite(h2.float()).all()
+
+
+@pytest.mark.slow
+def test_ramp_prefill_step_by_step_against_the_oracle():
+    # arc_recurrent_prefill(T = 16, k_low = 12) at the recurrent workload's size, one step at a
+    # time: each step runs through the schedule driver with T = 1 and must equal the same step
+    # composed from the individual calls, each of which is checked teacher-forced against the
+    # oracle on the GPU's own input of that step (NVFP4 + ARC steps 0..11, BF16 steps 12..15).
+    # Finally the whole T = 16 driver call must equal the chain of single steps.
+    c = W.RECURRENT
+    T, k_low = c["T"], 12
+    rec, h0, subs = make_block(S=c["S"], d=c["d"], ffn=c["ffn"], r=c["r"])
+    blk = arc.RecurrentBlock(c["d"], c["ffn"], EPS, [{k: v for k, v in s.items() if k != "bits"} for s in subs])
+    rows = sample_rows(c["S"], n=16, seed=2)
+    h = h0.clone()
+    for t in range(T):
+        low = t < k_low
+        h_drv = arc.recurrent_prefill_schedule(h.clone(), blk, [1 if low else 0])
+        hc = h.clone()
+        for L in subs:
+            hc = nvfp4_sublayer_teacher_forced(hc, L, c["r"], rows=rows) if low else \
+                bf16_sublayer_teacher_forced(hc, L, rows=rows)
+        torch.cuda.synchronize()
+        assert torch.equal(h_drv, hc), f"step {t}"
+        h = h_drv
+    h_full = arc.recurrent_prefill(h0.clone(), blk, T, k_low)
+    torch.cuda.synchronize()
+    assert arc.last_device_status() == 0
+    assert torch.equal(h_full, h)
+
+
+def add_fp8_weights(subs):
+    for L in subs:
+        L["gu_f8"] = arc.quantize_fp8(L["wgu"])
+        L["d_f8"] = arc.quantize_fp8(L["wd"])
+    torch.cuda.synchronize()
+    return subs
+
+
+def fp8_sublayer_teacher_forced(h, L, rows=None):
+    # RAMP's FP8 W8A8 step: RMSNorm (BF16), dynamic per-tensor FP8 activations, FP8 weights
+    S, d = h.shape
+    hb = to_bits(h)
+    n = arc.rmsnorm_bf16(h, L["gain"], EPS)
+    n_bits = to_bits(n)
+    np.testing.assert_array_equal(n_bits, O.rmsnorm(hb, to_bits(L["gain"]), float(np.float32(EPS))))
+    qa = arc.quantize_fp8(n)
+    sa = O.fp8_scale(O.amax(n_bits))
+    ca = O.quantize_fp8(n_bits, sa)
+    torch.cuda.synchronize()
+    assert qa.scale.item() == np.float32(sa)
+    np.testing.assert_array_equal(qa.codes.cpu().numpy(), ca)
+    wgu_bits = to_bits(L["wgu"])
+    sw = O.fp8_scale(O.amax(wgu_bits))
+    cw = O.quantize_fp8(wgu_bits, sw)
+    np.testing.assert_array_equal(L["gu_f8"].codes.cpu().numpy(), cw)
+    gu = arc.gemm_fp8(qa, L["gu_f8"])
+    rows = sample_rows(S) if rows is None else rows
+    ref = O.gemm_fp8_f64(ca, sa, cw, sw, rows=rows)
+    gu_bits = to_bits(gu)
+    assert normalized_gemm_error(gu_bits[rows], ref, row_norms(n_bits[rows]), row_norms(wgu_bits)) <= GEMM_TOL
+    act = arc.silu_mul_bf16(gu)
+    act_bits = to_bits(act)
+    silu_within_one_ulp(act_bits, gu_bits)
+    qd = arc.quantize_fp8(act)
+    s2 = O.fp8_scale(O.amax(act_bits))
+    c2 = O.quantize_fp8(act_bits, s2)
+    torch.cuda.synchronize()
+    assert qd.scale.item() == np.float32(s2)
+    np.testing.assert_array_equal(qd.codes.cpu().numpy(), c2)
+    wd_bits = to_bits(L["wd"])
+    swd = O.fp8_scale(O.amax(wd_bits))
+    cwd = O.quantize_fp8(wd_bits, swd)
+    h_new = arc.gemm_fp8(qd, L["d_f8"], out=h.clone(), add=h)
+    ref = O.gemm_fp8_f64(c2, s2, cwd, swd, rows=rows) + O.bf16_bits_to_f32(hb[rows])
+    assert normalized_gemm_error(to_bits(h_new)[rows], ref, row_norms(act_bits[rows]), row_norms(wd_bits),
+                                 with_add=True) <= GEMM_TOL
+    return h_new
+
+
+def _block(d, ffn, subs, beta=1.0):
+    return arc.RecurrentBlock(d, ffn, EPS, [{k: v for k, v in s.items() if k != "bits"} for s in subs], beta)
+
+
+def test_fp8_steps_teacher_forced_and_mixed_schedules():
+    # the driver's FP8 step equals the FP8 calls composed, each checked against the oracle; a
+    # schedule mixing all three formats equals its steps run one at a time
+    rec, h0, subs = make_block(S=200, d=512, ffn=1024, r=32)
+    add_fp8_weights(subs)
+    blk = _block(512, 1024, subs)
+    h_drv = arc.recurrent_prefill_schedule(h0.clone(), blk, [arc.STEP_FP8])
+    hc = h0.clone()
+    for L in subs:
+        hc = fp8_sublayer_teacher_forced(hc, L)
+    torch.cuda.synchronize()
+    assert torch.equal(h_drv, hc)
+    sched = [arc.STEP_FP8, arc.STEP_NVFP4, arc.STEP_BF16, arc.STEP_FP8, arc.STEP_BF16]
+    h_all = arc.recurrent_prefill_schedule(h0.clone(), blk, sched)
+    h = h0.clone()
+    for f in sched:
+        arc.recurrent_prefill_schedule(h, blk, [f])
+    torch.cuda.synchronize()
+    assert arc.last_device_status() == 0
+    assert torch.equal(h_all, h)
+
+
+def test_schedule_rejects_unknown_formats_and_missing_fp8_weights():
+    rec, h0, subs = make_block(S=64, d=256, ffn=512, r=32)
+    blk = _block(256, 512, subs)  # no FP8 weights
+    with pytest.raises(arc.ArcError):
+        arc.recurrent_prefill_schedule(h0.clone(), blk, [arc.STEP_BF16, arc.STEP_FP8])
+    with pytest.raises(arc.ArcError):
+        arc.recurrent_prefill_schedule(h0.clone(), blk, [3])
+    with pytest.raises(arc.ArcError):
+        _ = arc.recurrent_prefill(h0.clone(), _block(256, 512, subs, beta=1.5), 1, 0)
+
+
+@pytest.mark.slow
+def test_ramp_fp8_instantiation_at_the_recurrent_workload_size():
+    # RAMP's FP8-BF16 instantiation in form (T = 32, K = 24: FP8 W8A8 steps, then BF16) at the
+    # recurrent workload's size: the first FP8 step and the first BF16 step after the switch are
+    # checked teacher-forced against the oracle, and the whole schedule must equal its steps run
+    # one at a time
+    c = W.RECURRENT
+    rec, h0, subs = make_block(S=c["S"], d=c["d"], ffn=c["ffn"], r=c["r"])
+    add_fp8_weights(subs)
+    blk = _block(c["d"], c["ffn"], subs)
+    rows = sample_rows(c["S"], n=32, seed=3)
+    T, K = 32, 24
+    sched = [arc.STEP_FP8] * K + [arc.STEP_BF16] * (T - K)
+    h = h0.clone()
+    for t, f in enumerate(sched):
+        if t in (0, K):
+            hc = h.clone()
+            for L in subs:
+                hc = fp8_sublayer_teacher_forced(hc, L, rows=rows) if f == arc.STEP_FP8 else \
+                    bf16_sublayer_teacher_forced(hc, L, rows=rows)
+        arc.recurrent_prefill_schedule(h, blk, [f])
+        if t in (0, K):
+            torch.cuda.synchronize()
+            assert torch.equal(h, hc), f"step {t}"
+    h_all = arc.recurrent_prefill_schedule(h0.clone(), blk, sched)
+    torch.cuda.synchronize()
+    assert arc.last_device_status() == 0
+    assert torch.equal(h_all, h)
+
+
+def test_damped_residual_block_equals_its_composed_calls():
+    # h <- beta h + F(h) with beta = 1/2: the residual term is scaled (exactly, by a power of
+    # two) before the down projection adds to it, in every format
+    beta = 0.5
+    rec, h0, subs = make_block(S=130, d=256, ffn=512, r=32)
+    add_fp8_weights(subs)
+    blk = _block(256, 512, subs, beta)
+    for f in (arc.STEP_NVFP4, arc.STEP_FP8, arc.STEP_BF16):
+        h_drv = arc.recurrent_prefill_schedule(h0.clone(), blk, [f])
+        h = h0.clone()
+        for L in subs:
+            if f == arc.STEP_NVFP4:
+                qa = arc.quantize_act_nvfp4(h, L["idx_gu"], rms_gain=L["gain"], eps=EPS)
+                act = arc.silu_mul_bf16(arc.gemm_nvfp4(qa, L["gu_q"]))
+                qd = arc.quantize_act_nvfp4(act, L["idx_d"])
+                hs = (h.float() * beta).bfloat16()
+                h = arc.gemm_nvfp4(qd, L["d_q"], out=hs, add=hs)
+            elif f == arc.STEP_FP8:
+                n = arc.rmsnorm_bf16(h, L["gain"], EPS)
+                act = arc.silu_mul_bf16(arc.gemm_fp8(arc.quantize_fp8(n), L["gu_f8"]))
+                hs = (h.float() * beta).bfloat16()
+                h = arc.gemm_fp8(arc.quantize_fp8(act), L["d_f8"], out=hs, add=hs)
+            else:
+                n = arc.rmsnorm_bf16(h, L["gain"], EPS)
+                act = arc.silu_mul_bf16(arc.gemm_bf16(n, L["wgu"]))
+                hs = (h.float() * beta).bfloat16()
+                h = arc.gemm_bf16(act, L["wd"], out=hs, add=hs)
+        torch.cuda.synchronize()
+        assert arc.last_device_status() == 0
+        assert torch.equal(h_drv, h), f

@@ -41,6 +41,22 @@ def _worker(rank, world, port, q):
             wsum = [torch.zeros_like(w) for _ in range(world)]
             torch.distributed.all_gather(wsum, w)
             out[workload] = (torch.cat(xs).numpy().astype(np.uint16), [t.tolist() for t in wsum])
+        # the replica scheme's quantization of this rank's own rows: the rank's tensor scale is the
+        # amax of its own shard; with one 4-byte all-reduce(max) of the amax the ranks would share
+        # the single-process scale instead
+        import oracle as O
+
+        d = W.llama8b("o", rows=M, row0=rank * M, w_rows=8)
+        idx = O.calibrate(W.llama8b("o", rows=2 * M, with_w=False)["x"], 32)
+        a_mine = O.amax(d["x"])
+        s_mine = O.tensor_scale(a_mine)
+        c_mine, sf_mine = O.quantize_act(d["x"], idx, s_mine)
+        a_all = torch.tensor([a_mine], dtype=torch.float64)
+        torch.distributed.all_reduce(a_all, op=torch.distributed.ReduceOp.MAX)
+        s_glob = O.tensor_scale(float(a_all.item()))
+        c_glob, sf_glob = O.quantize_act(d["x"], idx, s_glob)
+        out["shard"] = dict(s_mine=s_mine, c_mine=c_mine, sf_mine=sf_mine, s_glob=s_glob, c_glob=c_glob,
+                            sf_glob=sf_glob, idx=idx)
         bench._barrier(world)
         q.put(out)
     finally:
@@ -68,6 +84,26 @@ def test_two_gloo_ranks():
         np.testing.assert_array_equal(gathered, gen())
         assert not np.array_equal(gathered[:8], gathered[8:])
         assert wsums[0] == wsums[1]  # the same weights on both ranks
+    # each rank's codes of its own rows equal the single-process oracle on the same rows with
+    # that rank's scale; with the all-reduced scale they equal the single-process quantization of
+    # the whole batch, row for row
+    import oracle as O
+
+    full = W.llama8b("o", rows=16, with_w=False)["x"]
+    idx = res[0]["shard"]["idx"]
+    s_one = O.tensor_scale(O.amax(full))
+    c_one, sf_one = O.quantize_act(full, idx, s_one)
+    for o in res:
+        sh, r0 = o["shard"], 8 * o["rank"]
+        c_rows, sf_rows = O.quantize_act(full[r0:r0 + 8], idx, sh["s_mine"])
+        np.testing.assert_array_equal(sh["c_mine"], c_rows)
+        np.testing.assert_array_equal(sh["sf_mine"], sf_rows)
+        assert sh["s_glob"] == s_one
+        np.testing.assert_array_equal(sh["c_glob"], c_one[r0:r0 + 8])
+        np.testing.assert_array_equal(sh["sf_glob"], sf_one[r0:r0 + 8])
+    # the per-rank scales differ from the whole batch's on at least one rank (the replica scheme
+    # does not reproduce the single-process scale bit for bit, and says so)
+    assert any(o["shard"]["s_mine"] != s_one for o in res)
 
 
 def test_value_is_the_whole_job_throughput():
@@ -84,3 +120,35 @@ def test_value_is_the_whole_job_throughput():
     assert two["n_gpus"] == 2 and two["scaling"] == "weak"
     flops = sum(bench.layer_flops(L) for L in layers)
     assert abs(one["value"] - flops * 10 / 6.4e-3 / 1e12) < 1e-9 * one["value"]
+
+
+def test_bench_launcher_refuses_more_gpus_than_visible():
+    # without a launcher, --gpus N starts one process per GPU; with fewer visible GPUs it refuses
+    import subprocess
+    import sys
+
+    if torch.cuda.device_count() >= 2:
+        return
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    p = subprocess.run([sys.executable, bench.__file__, "--gpus", "2", "--steps", "1", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=300, env=env)
+    assert p.returncode == 2
+    assert "CUDA device(s) are visible" in p.stderr
+
+
+def test_spawned_rank_environment(monkeypatch):
+    # a spawned rank sees the rendezvous torchrun would give it
+    seen = {}
+
+    def fake_run(args, ap):
+        seen.update({k: os.environ[k] for k in ("RANK", "LOCAL_RANK", "WORLD_SIZE", "MASTER_ADDR", "MASTER_PORT")})
+
+    class A:
+        gpus = 4
+
+    for k in ("RANK", "LOCAL_RANK", "WORLD_SIZE", "MASTER_ADDR", "MASTER_PORT"):
+        monkeypatch.delenv(k, raising=False)
+    monkeypatch.setattr(bench, "run", fake_run)
+    bench._rank_main(3, A, 29555)
+    assert seen == {"RANK": "3", "LOCAL_RANK": "3", "WORLD_SIZE": "4", "MASTER_ADDR": "127.0.0.1",
+                    "MASTER_PORT": "29555"}
