@@ -544,16 +544,18 @@ def contractive_study(arc, device, stream, S=1024, d=2048, F=8192, T=16, budget=
                       n_random=24):
     """RAMP's placement result (section 3, Theorem 3.2: with locally contractive steps, low
     precision early and BF16 late minimises the final-error bound; late placement maximises it;
-    random schedules fall between) checked on a block built to contract: the damped residual
-    h <- beta h + F(h) with beta = 1/2 and RMSNorm eps = 1 (n is then close to linear in h), the
-    recurrent workload's weights. The contraction factor is measured (BF16 step map, the ratio of
-    output to input perturbation norms); each schedule's final hidden-state error is against the
-    all-BF16 run. Fidelity only: nothing here is timed."""
+    random schedules fall between) checked on a block built to contract towards a nonzero fixed
+    point: the damped residual with input injection h <- beta h + e + F(h), beta = 1/2, e ~ N(0, 1)
+    (a recurrence that re-reads its input every step), RMSNorm eps = 1, the recurrent workload's
+    weights. The contraction factor is measured (BF16 step map, the ratio of output to input
+    perturbation norms); each schedule's final hidden-state error is against the all-BF16 run.
+    Fidelity only: nothing here is timed."""
     import workloads as W
 
     rec = W.recurrent(S=S, d=d, ffn=F)
     with torch.cuda.stream(stream):
         h0 = W.to_torch_bf16(rec["h"]).to(device)
+        e = W.to_torch_bf16(W.matrix_bf16(W.RECURRENT["seed"], 99, S, d, 1.0)).to(device)
         subs = []
         for L in rec["layers"]:
             wgu, wd, gain = (W.to_torch_bf16(L[k]).to(device) for k in ("wgu", "wd", "gain"))
@@ -564,7 +566,7 @@ def contractive_study(arc, device, stream, S=1024, d=2048, F=8192, T=16, budget=
             subs.append(dict(gain=gain, wgu=wgu, wd=wd, idx_gu=idx_gu, idx_d=idx_d,
                              gu_q=arc.pack_weight_nvfp4(wgu, idx_gu, stream=stream),
                              d_q=arc.pack_weight_nvfp4(wd, idx_d, stream=stream)))
-        blk = arc.RecurrentBlock(d, F, eps, subs, beta)
+        blk = arc.RecurrentBlock(d, F, eps, subs, beta, inject=e)
         ws = torch.empty(blk.workspace_bytes(S), dtype=torch.uint8, device=device)
 
         def run(flags, h_in=None):
@@ -604,8 +606,8 @@ def contractive_study(arc, device, stream, S=1024, d=2048, F=8192, T=16, budget=
     stream.synchronize()
     if arc.last_device_status(stream) != 0:
         raise RuntimeError("device status set during the contractive study")
-    return {"block": f"damped residual beta={beta}, RMSNorm eps={eps}, S={S}, d={d}, ffn={F}, r={r}, T={T}, "
-                     f"{budget} NVFP4 + {k} BF16 steps",
+    return {"block": f"damped residual with input injection (h <- beta h + e + F(h)), beta={beta}, e~N(0,1), "
+                     f"RMSNorm eps={eps}, S={S}, d={d}, ffn={F}, r={r}, T={T}, {budget} NVFP4 + {k} BF16 steps",
             "contraction_factor": {"median": statistics.median(rho), "max": max(rho)},
             "schedules": out,
             "random": {"n": n_random, "min": min(rerr), "median": statistics.median(rerr), "max": max(rerr)},

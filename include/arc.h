@@ -299,8 +299,9 @@ arc_status arc_silu_mul_bf16(const void* gu_bf16, int64_t S, int64_t F, int64_t 
 /* ----------------------------------------------------------------------------------------- */
 
 /*
- * One pre-norm SwiGLU residual sublayer: h <- beta h + W_down (silu(W_g n) * (W_u n)),
- * n = RMSNorm(h)*g, beta = the block's residual_scale. All pointers are device pointers. The
+ * One pre-norm SwiGLU residual sublayer: h <- beta h + e + W_down (silu(W_g n) * (W_u n)),
+ * n = RMSNorm(h)*g, beta and e = the block's residual_scale and inject_bf16 (1 and none for the
+ * plain block); beta h + e is rounded to bf16 before the down projection adds to it. All pointers are device pointers. The
  * NVFP4 fields are the arc_pack_weight_nvfp4 outputs of the same weights augmented with
  * idx_gateup (channels of n, in [0, d)) and idx_down (channels of the SwiGLU output, in
  * [0, ffn)). The FP8 fields are the arc_quantize_fp8 outputs of the same weights (codes with row
@@ -333,9 +334,13 @@ typedef struct {
   float eps;      /* RMSNorm epsilon */
   int32_t n_sublayers;
   const arc_swiglu_sublayer* sublayers; /* host array of n_sublayers entries */
-  float residual_scale; /* beta in (0, 1] of the damped residual h <- beta h + F(h); 0 or 1 is the
-                           plain residual block. beta < 1 makes the step map contractive when F
-                           is small, the regime of RAMP's error analysis (section 3). */
+  float residual_scale; /* beta in (0, 1] of the damped residual h <- beta h + e + F(h); 0 or 1 is
+                           the plain residual block */
+  const void* inject_bf16; /* e: device bf16 [S, d] (row stride d) added to the damped residual of
+                              every sublayer, or NULL. With beta < 1 and a small F the step map
+                              contracts towards a fixed point that e keeps away from zero: the
+                              regime of RAMP's error analysis (section 3, local contraction of a
+                              recurrence that re-reads its input at every step). */
 } arc_swiglu_block;
 
 /* Workspace of arc_recurrent_prefill for S tokens. */
@@ -388,7 +393,9 @@ arc_status arc_set_wait_limit_ns(uint64_t ns);
 /*
  * Failure-injection switch for tests (0 = off). 1: the next arc_gemm_* launch withholds its
  * first operand load, so its consumer's bounded wait must run out and report ARC_ERR_TIMEOUT.
- * The switch resets itself after one launch.
+ * 2: the next reordered quantization (arc_quantize_act_nvfp4_reordered or
+ * arc_pack_weight_nvfp4_reordered) withholds the first row copy of its first CTA, with the same
+ * outcome. The switch resets itself after the launch it applies to.
  */
 arc_status arc_debug_inject(int32_t kind);
 

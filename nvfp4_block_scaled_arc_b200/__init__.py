@@ -44,7 +44,7 @@ class SwigluSublayer(ctypes.Structure):
 class SwigluBlock(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int64), ("ffn", ctypes.c_int64), ("eps", ctypes.c_float),
                 ("n_sublayers", ctypes.c_int32), ("sublayers", ctypes.POINTER(SwigluSublayer)),
-                ("residual_scale", ctypes.c_float)]
+                ("residual_scale", ctypes.c_float), ("inject_bf16", ctypes.c_void_p)]
 
 
 STEP_BF16, STEP_NVFP4, STEP_FP8 = 0, 1, 2  # per-step formats of arc_recurrent_prefill_schedule
@@ -351,9 +351,11 @@ class RecurrentBlock:
     """Host description of the shared SwiGLU block (keeps the ctypes structs and tensors alive).
     Each sublayer dict holds gain, wgu, wd (bf16), gu_q, d_q (packed NVFP4 weights), idx_gu,
     idx_d, and optionally gu_f8, d_f8 (FP8Tensor weights, needed by FP8 steps).
-    residual_scale is the damped residual's beta (1: the plain residual block)."""
+    residual_scale is the damped residual's beta and inject an optional bf16 [S, d] term e added to
+    it (h <- beta h + e + F(h); 1 and None: the plain residual block)."""
 
-    def __init__(self, d: int, ffn: int, eps: float, sublayers: list[dict], residual_scale: float = 1.0):
+    def __init__(self, d: int, ffn: int, eps: float, sublayers: list[dict], residual_scale: float = 1.0,
+                 inject: torch.Tensor | None = None):
         self.d, self.ffn, self.eps = d, ffn, eps
         self.sub = sublayers
         arr = (SwigluSublayer * len(sublayers))()
@@ -367,7 +369,9 @@ class RecurrentBlock:
                 f8g.codes.data_ptr() if f8g is not None else None, f8g.scale.data_ptr() if f8g is not None else None,
                 f8d.codes.data_ptr() if f8d is not None else None, f8d.scale.data_ptr() if f8d is not None else None)
         self._arr = arr
-        self.block = SwigluBlock(d, ffn, float(eps), len(sublayers), arr, float(residual_scale))
+        self._inject = inject
+        self.block = SwigluBlock(d, ffn, float(eps), len(sublayers), arr, float(residual_scale),
+                                 inject.data_ptr() if inject is not None else None)
 
     def workspace_bytes(self, S: int) -> int:
         return int(lib().arc_recurrent_workspace_bytes(S, ctypes.byref(self.block)))

@@ -60,10 +60,11 @@ __global__ void __launch_bounds__(256) k_silu_mul(const __nv_bfloat16* __restric
   }
 }
 
-// h[m, k] = bf16(beta * h[m, k]) in place, 8 values per thread (d % 8 == 0): the damped residual
-// of a contractive recurrent block, applied before the sublayer's residual add.
-__global__ void __launch_bounds__(256) k_scale_bf16(__nv_bfloat16* __restrict__ h, int64_t ldh, int M, int d,
-                                                    float beta) {
+// h[m, k] = bf16(fp32(beta * h[m, k]) + e[m, k]) in place (e optional), 8 values per thread
+// (d % 8 == 0): the damped residual (with input injection) of a contractive recurrent block,
+// applied before the sublayer's residual add.
+__global__ void __launch_bounds__(256) k_damp_bf16(__nv_bfloat16* __restrict__ h, int64_t ldh, int M, int d,
+                                                   float beta, const __nv_bfloat16* __restrict__ e) {
   const int vpr = d >> 3;
   const int64_t total = static_cast<int64_t>(M) * vpr;
   for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < total;
@@ -72,10 +73,14 @@ __global__ void __launch_bounds__(256) k_scale_bf16(__nv_bfloat16* __restrict__ 
     const int j = static_cast<int>(v - m * vpr) * 8;
     uint4* p = reinterpret_cast<uint4*>(h + m * ldh + j);
     const uint4 w = *p;
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    const uint4 ew = e ? ld_nc_v4(e + m * d + j) : make_uint4(0, 0, 0, 0);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w}, es[4] = {ew.x, ew.y, ew.z, ew.w};
     uint32_t o[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) o[i] = pack_bf16x2_rn(__fmul_rn(beta, bf16_lo(ws[i])), __fmul_rn(beta, bf16_hi(ws[i])));
+    for (int i = 0; i < 4; ++i) {
+      const float lo = __fmul_rn(beta, bf16_lo(ws[i])), hi = __fmul_rn(beta, bf16_hi(ws[i]));
+      o[i] = e ? pack_bf16x2_rn(__fadd_rn(lo, bf16_lo(es[i])), __fadd_rn(hi, bf16_hi(es[i]))) : pack_bf16x2_rn(lo, hi);
+    }
     *p = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }

@@ -131,11 +131,12 @@ bool make_store_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t o
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int take_inject() {
+// The armed failure injection if it is of this kind (it is then disarmed), else 0.
+int take_inject(int kind) {
   std::lock_guard<std::mutex> lk(g_mu);
-  const int k = g_inject;
+  if (g_inject != kind) return 0;
   g_inject = 0;
-  return k;
+  return kind;
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -236,6 +237,7 @@ arc_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, con
   a.sf = sf;
   a.dup = dup;
   a.wait_ns = g_wait_ns;
+  a.inject = perm ? take_inject(2) : 0;
   const int mpad = static_cast<int>((M + 127) / 128 * 128);
   // the second launch may begin while the first one runs; it waits for the first one's results
   cudaLaunchAttribute pdl[1];
@@ -510,7 +512,7 @@ arc_status arc_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_sf, const flo
       !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b_codes, static_cast<uint64_t>(kpad / 2),
                 static_cast<uint64_t>(N), static_cast<uint64_t>(kpad / 2), 128, g.box_rows_b))
     return ARC_ERR_CUDA;
-  g.inject = take_inject();
+  g.inject = take_inject(1);
   return gemm_launch<arc::kGemmFP4>(ta, tb, g, sms, add_bf16 != nullptr, S(stream));
 }
 
@@ -563,7 +565,7 @@ arc_status arc_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_sf, const uin
       !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b_codes, static_cast<uint64_t>(kpad / 2),
                 static_cast<uint64_t>(N), static_cast<uint64_t>(kpad / 2), 128, g.box_rows_b))
     return ARC_ERR_CUDA;
-  g.inject = take_inject();
+  g.inject = take_inject(1);
   return gemm_launch<arc::kGemmMX4>(ta, tb, g, sms, add_bf16 != nullptr, S(stream));
 }
 
@@ -600,7 +602,7 @@ arc_status arc_gemm_bf16(const void* x_bf16, int64_t ldx, const void* w_bf16, in
       !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_bf16, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
                 static_cast<uint64_t>(ldw * 2), 64, g.box_rows_b))
     return ARC_ERR_CUDA;
-  g.inject = take_inject();
+  g.inject = take_inject(1);
   return gemm_launch<arc::kGemmBF16>(ta, tb, g, sms, add_bf16 != nullptr, S(stream));
 }
 
@@ -679,7 +681,7 @@ arc_status arc_gemm_fp8(const uint8_t* a_codes, int64_t lda, const float* d_a_sc
       !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b_codes, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
                 static_cast<uint64_t>(ldb), 128, g.box_rows_b))
     return ARC_ERR_CUDA;
-  g.inject = take_inject();
+  g.inject = take_inject(1);
   return gemm_launch<arc::kGemmFP8>(ta, tb, g, sms, add_bf16 != nullptr, S(stream));
 }
 
@@ -745,12 +747,13 @@ size_t arc_recurrent_workspace_bytes(int64_t S_, const arc_swiglu_block* blk) {
   return off[6] + arc_quantize_workspace_bytes(S_, rmax);
 }
 
-// h = bf16(beta * h), the damped residual of a contractive block.
-static arc_status scale_bf16(void* h, int64_t S_, int64_t d, float beta, arc_stream_t stream, int sms) {
+// h = bf16(beta * h + e), the damped residual (with input injection) of a contractive block.
+static arc_status damp_bf16(void* h, int64_t S_, int64_t d, float beta, const void* e, arc_stream_t stream, int sms) {
   const int64_t vecs = S_ * (d / 8);
   const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((vecs + 255) / 256, static_cast<int64_t>(sms) * 8));
-  arc::k_scale_bf16<<<static_cast<unsigned>(blocks), 256, 0, S(stream)>>>(static_cast<__nv_bfloat16*>(h), d,
-                                                                         static_cast<int>(S_), static_cast<int>(d), beta);
+  arc::k_damp_bf16<<<static_cast<unsigned>(blocks), 256, 0, S(stream)>>>(
+      static_cast<__nv_bfloat16*>(h), d, static_cast<int>(S_), static_cast<int>(d), beta,
+      static_cast<const __nv_bfloat16*>(e));
   return launch_status();
 }
 
@@ -774,8 +777,11 @@ arc_status recurrent_run(void* h_bf16, int64_t S_, const arc_swiglu_block* blk, 
         if (!L.gateup_fp8 || !L.gateup_fp8_scale || !L.down_fp8 || !L.down_fp8_scale) return ARC_ERR_INVALID_ARG;
       }
   }
+  const void* inj = blk->inject_bf16;
+  if (inj && (reinterpret_cast<uintptr_t>(inj) & 15u)) return ARC_ERR_ALIGNMENT;
+  const bool damp = beta != 1.0f || inj != nullptr;
   int sms = 0;
-  if (beta != 1.0f) {
+  if (damp) {
     const arc_status dc = device_check(&sms);
     if (dc != ARC_OK) return dc;
   }
@@ -809,7 +815,7 @@ arc_status recurrent_run(void* h_bf16, int64_t S_, const arc_swiglu_block* blk, 
         if ((st = arc_quantize_act_nvfp4(act, S_, F, F, L.idx_down, L.r_down, nullptr, 0.0f, nullptr, codes, sf,
                                          sA + 1, qws, qws_bytes, stream)) != ARC_OK)
           return st;
-        if (beta != 1.0f && (st = scale_bf16(h_bf16, S_, d, beta, stream, sms)) != ARC_OK) return st;
+        if (damp && (st = damp_bf16(h_bf16, S_, d, beta, inj, stream, sms)) != ARC_OK) return st;
         if ((st = arc_gemm_nvfp4(codes, sf, sA + 1, L.down_codes, L.down_sf, L.down_scale, S_, d, F + L.r_down,
                                  h_bf16, d, h_bf16, d, stream)) != ARC_OK)
           return st;
@@ -822,7 +828,7 @@ arc_status recurrent_run(void* h_bf16, int64_t S_, const arc_swiglu_block* blk, 
         if ((st = arc_silu_mul_bf16(gu, S_, F, 2 * F, act, F, stream)) != ARC_OK) return st;
         if ((st = arc_quantize_fp8(act, S_, F, F, nullptr, codes, F, sA + 1, qws, qws_bytes, stream)) != ARC_OK)
           return st;
-        if (beta != 1.0f && (st = scale_bf16(h_bf16, S_, d, beta, stream, sms)) != ARC_OK) return st;
+        if (damp && (st = damp_bf16(h_bf16, S_, d, beta, inj, stream, sms)) != ARC_OK) return st;
         if ((st = arc_gemm_fp8(codes, F, sA + 1, L.down_fp8, F, L.down_fp8_scale, S_, d, F, h_bf16, d, h_bf16, d,
                                stream)) != ARC_OK)
           return st;
@@ -831,7 +837,7 @@ arc_status recurrent_run(void* h_bf16, int64_t S_, const arc_swiglu_block* blk, 
         if ((st = arc_gemm_bf16(nrm, d, L.w_gateup_bf16, d, S_, 2 * F, d, gu, 2 * F, nullptr, 0, stream)) != ARC_OK)
           return st;
         if ((st = arc_silu_mul_bf16(gu, S_, F, 2 * F, act, F, stream)) != ARC_OK) return st;
-        if (beta != 1.0f && (st = scale_bf16(h_bf16, S_, d, beta, stream, sms)) != ARC_OK) return st;
+        if (damp && (st = damp_bf16(h_bf16, S_, d, beta, inj, stream, sms)) != ARC_OK) return st;
         if ((st = arc_gemm_bf16(act, F, L.w_down_bf16, F, S_, d, F, h_bf16, d, h_bf16, d, stream)) != ARC_OK)
           return st;
       }
@@ -915,7 +921,7 @@ arc_status arc_quantize_act_nvfp4_static_scratch(const void* x_bf16, int64_t M, 
 }
 
 arc_status arc_debug_inject(int32_t kind) {
-  if (kind < 0 || kind > 1) return ARC_ERR_INVALID_ARG;
+  if (kind < 0 || kind > 2) return ARC_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lk(g_mu);
   g_inject = kind;
   return ARC_OK;

@@ -53,6 +53,7 @@ struct QuantArgs {
   uint8_t* sf;
   int dup;       // 1: weights (stash the value itself), 0: activations (stash the residual)
   uint64_t wait_ns;  // bound on the reordered kernel's waits (one that runs out sets the timeout status)
+  int inject;        // 2: CTA 0 withholds its first row copy (failure-injection test of the bounded waits)
 };
 
 // Read-only 16-byte load that allocates in L1: two lanes' loads of one 32-byte sector then
@@ -878,6 +879,7 @@ __global__ void __launch_bounds__(kQReoThreads, 3) k_quant_reordered(QuantArgs a
     const int buf = it & 1;
     const uint32_t bytes = static_cast<uint32_t>(a.K) * 2u;
     mbar_arrive_expect_tx(&row_full[buf], bytes);
+    if (a.inject == 2 && blockIdx.x == 0 && it == 0) return;  // withheld: the wait for it must run out
     bulk_load(qreo_smem + buf * rowb, a.x + m * a.ldx, bytes, &row_full[buf]);
     armed |= 1u << buf;
   };

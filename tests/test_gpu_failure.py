@@ -37,3 +37,25 @@ def test_withheld_load_times_out_and_recovers(kind):
     torch.cuda.synchronize()
     assert arc.last_device_status() == 0
     assert torch.equal(again, good)
+
+
+def test_withheld_row_copy_in_the_reordered_quantizer_times_out_and_recovers():
+    # the reordered quantizer stages rows by bulk copies with bounded waits: a copy that never
+    # comes must end in ARC_ERR_TIMEOUT, not a hang, and leave the context usable
+    d = W.llama8b("o", rows=300, with_w=False)
+    x = to_dev(d["x"])
+    perm = arc.calibrate_order(x)
+    good = arc.quantize_act_nvfp4_reordered(x, perm, 128)
+    torch.cuda.synchronize()
+    assert arc.last_device_status() == 0
+    arc.set_wait_limit_ns(50_000_000)  # 50 ms
+    try:
+        arc.debug_inject(2)
+        arc.quantize_act_nvfp4_reordered(x, perm, 128)
+        assert arc.last_device_status() == TIMEOUT
+    finally:
+        arc.set_wait_limit_ns(2_000_000_000)
+    again = arc.quantize_act_nvfp4_reordered(x, perm, 128)
+    torch.cuda.synchronize()
+    assert arc.last_device_status() == 0
+    assert torch.equal(again.codes, good.codes) and torch.equal(again.sf, good.sf)

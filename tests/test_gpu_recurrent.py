@@ -282,8 +282,8 @@ def fp8_sublayer_teacher_forced(h, L, rows=None):
     return h_new
 
 
-def _block(d, ffn, subs, beta=1.0):
-    return arc.RecurrentBlock(d, ffn, EPS, [{k: v for k, v in s.items() if k != "bits"} for s in subs], beta)
+def _block(d, ffn, subs, beta=1.0, inject=None):
+    return arc.RecurrentBlock(d, ffn, EPS, [{k: v for k, v in s.items() if k != "bits"} for s in subs], beta, inject)
 
 
 def test_fp8_steps_teacher_forced_and_mixed_schedules():
@@ -349,13 +349,19 @@ def test_ramp_fp8_instantiation_at_the_recurrent_workload_size():
     assert torch.equal(h_all, h)
 
 
-def test_damped_residual_block_equals_its_composed_calls():
-    # h <- beta h + F(h) with beta = 1/2: the residual term is scaled (exactly, by a power of
-    # two) before the down projection adds to it, in every format
+@pytest.mark.parametrize("with_inject", [False, True])
+def test_damped_residual_block_equals_its_composed_calls(with_inject):
+    # h <- beta h + e + F(h) with beta = 1/2: the residual term bf16(fp32(beta h) + e) is formed
+    # before the down projection adds to it, in every format
     beta = 0.5
     rec, h0, subs = make_block(S=130, d=256, ffn=512, r=32)
     add_fp8_weights(subs)
-    blk = _block(256, 512, subs, beta)
+    e = to_dev(W.matrix_bf16(5, 9, 130, 256, 1.0)) if with_inject else None
+    blk = _block(256, 512, subs, beta, e)
+
+    def damp(h):
+        return (h.float() * beta + (e.float() if e is not None else 0.0)).bfloat16()
+
     for f in (arc.STEP_NVFP4, arc.STEP_FP8, arc.STEP_BF16):
         h_drv = arc.recurrent_prefill_schedule(h0.clone(), blk, [f])
         h = h0.clone()
@@ -364,18 +370,19 @@ def test_damped_residual_block_equals_its_composed_calls():
                 qa = arc.quantize_act_nvfp4(h, L["idx_gu"], rms_gain=L["gain"], eps=EPS)
                 act = arc.silu_mul_bf16(arc.gemm_nvfp4(qa, L["gu_q"]))
                 qd = arc.quantize_act_nvfp4(act, L["idx_d"])
-                hs = (h.float() * beta).bfloat16()
+                hs = damp(h)
                 h = arc.gemm_nvfp4(qd, L["d_q"], out=hs, add=hs)
             elif f == arc.STEP_FP8:
                 n = arc.rmsnorm_bf16(h, L["gain"], EPS)
                 act = arc.silu_mul_bf16(arc.gemm_fp8(arc.quantize_fp8(n), L["gu_f8"]))
-                hs = (h.float() * beta).bfloat16()
+                hs = damp(h)
                 h = arc.gemm_fp8(arc.quantize_fp8(act), L["d_f8"], out=hs, add=hs)
             else:
                 n = arc.rmsnorm_bf16(h, L["gain"], EPS)
                 act = arc.silu_mul_bf16(arc.gemm_bf16(n, L["wgu"]))
-                hs = (h.float() * beta).bfloat16()
+                hs = damp(h)
                 h = arc.gemm_bf16(act, L["wd"], out=hs, add=hs)
         torch.cuda.synchronize()
         assert arc.last_device_status() == 0
         assert torch.equal(h_drv, h), f
+
