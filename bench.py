@@ -17,14 +17,19 @@ Other workloads (--workload), same timing rules:
              applied T = 16 times to H [4096, 2048]: one prefill per k_low in {0, 8, 12, 16}
              (steps before k_low in NVFP4 + ARC with r = 64, the rest BF16); time per prefill,
              speedup against k_low = 0 and the hidden-state error against all-BF16; after the
-             timed region, a schedule study at 12 of 16 NVFP4 steps (RAMP's order, BF16 first,
-             interleaved, random placements): error and time of each
+             timed region: a schedule study at 12 of 16 NVFP4 steps (RAMP's order, BF16 first,
+             interleaved, random placements), RAMP's own T = 32 / K = 24 instantiation with FP8
+             W8A8 steps next to NVFP4 + ARC steps, and the placement study on a block built to
+             contract (measured contraction factor; RAMP order vs Early-BF16 vs 24 random)
 
 Variants of the linear-layer workloads:
   --reorder      channels reordered by calibration abs-max before the primary quantization
                  (the outlier set is the first r of the order); adds the error against BF16
   --format fp8   FP8 W8A8 with per-tensor scales instead of NVFP4 + ARC (metric: FP8 GEMM
                  TFLOP/s against 2 x the measured BF16 peak); adds the error against BF16
+  --format mxfp4 MXFP4 with augmented residual channels (E2M1 codes, one power-of-two E8M0 scale
+                 per 32 values, no tensor scale: the quantizer is one pass over X); adds the
+                 error against BF16
 
 Metric: NVFP4 ARC GEMM TFLOP/s = sum over the step of 2*M*N*(K+r) / step time, with the fused
 activation quantizer's GB/s (read X + write codes + scale bytes) beside it.
@@ -475,7 +480,8 @@ def run_recurrent(args, rank, world, device):
             idx_d = arc.calibrate_outliers(act, r, stream=stream)
             subs.append(dict(gain=gain, wgu=wgu, wd=wd, idx_gu=idx_gu, idx_d=idx_d,
                              gu_q=arc.pack_weight_nvfp4(wgu, idx_gu, stream=stream),
-                             d_q=arc.pack_weight_nvfp4(wd, idx_d, stream=stream)))
+                             d_q=arc.pack_weight_nvfp4(wd, idx_d, stream=stream),
+                             gu_f8=arc.quantize_fp8(wgu, stream=stream), d_f8=arc.quantize_fp8(wd, stream=stream)))
         blk = arc.RecurrentBlock(d, F, eps, subs)
         wsp = torch.empty(blk.workspace_bytes(S), dtype=torch.uint8, device=device)
         h = torch.empty_like(h0)
@@ -533,8 +539,11 @@ def run_recurrent(args, rank, world, device):
                              "gemm_tflops": fl / (ms[k] * 1e-3) / 1e12,
                              "hidden_state_rel_err_vs_all_bf16": fidelity[k]}
     kk = 12 if 12 in ms else k_lows[-1]
-    study = schedule_study(arc, h, h0, blk, wsp, flush, stream, T, kk, out[0], device)
-    contractive = contractive_study(arc, device, stream, T=T, budget=kk, r=r)
+    study = ramp_fp8 = contractive = None
+    if not args.no_studies:
+        study = schedule_study(arc, h, h0, blk, wsp, flush, stream, T, kk, out[0], device)
+        ramp_fp8 = ramp_instantiations(arc, h, h0, blk, wsp, flush, stream, device)
+        contractive = contractive_study(arc, device, stream, T=T, budget=kk, r=r)
     # kernels per prefill: NVFP4 step = 2 x (2 quantizer launches + GEMM + SiLU + 2 quantizer
     # launches + GEMM), BF16 step = 2 x (RMSNorm + GEMM + SiLU + GEMM)
     launches = args.steps * sum(k * 2 * 7 + (T - k) * 2 * 4 for k in k_lows)
@@ -547,7 +556,8 @@ def run_recurrent(args, rank, world, device):
         "config": {"workload": f"recurrent SwiGLU block: S={S}, d={d}, ffn={F}, 2 pre-norm sublayers, T={T}, "
                                f"k_low in {k_lows}, r={r}",
                    "l2": "flushed before every prefill (256 MiB written, then read back)", "parallelism": f"replicas x{world}"},
-        "per_k_low": per, "schedule_study": study, "contractive_study": contractive, "clocks": clk.summary(),
+        "per_k_low": per, "schedule_study": study, "ramp_t32_k24": ramp_fp8, "contractive_study": contractive,
+        "clocks": clk.summary(),
         "e2e": None, "gpu_launches": launches,
     }
 
@@ -626,6 +636,43 @@ def contractive_study(arc, device, stream, S=1024, d=2048, F=8192, T=16, budget=
             "schedules": out,
             "random": {"n": n_random, "min": min(rerr), "median": statistics.median(rerr), "max": max(rerr)},
             "ordering_holds": out["ramp"]["err"] <= min(rerr) and max(rerr) <= out["early_bf16"]["err"]}
+
+
+def ramp_instantiations(arc, h, h0, blk, wsp, flush, stream, device, T=32, K=24, reps=5):
+    """RAMP's own instantiation ("RAMP…" §4.2: T = 32 recurrent steps, the first K = 24 in FP8 W8A8
+    with dynamic per-tensor FP8 activations, the last 8 in BF16) next to the same schedule with
+    NVFP4 + ARC low-precision steps and the all-BF16 prefill: prefill time (median of reps, L2
+    flushed before each) and final hidden-state error against all-BF16. Run after the timed
+    region."""
+    sch = {"all_bf16": [arc.STEP_BF16] * T,
+           "ramp_fp8": [arc.STEP_FP8] * K + [arc.STEP_BF16] * (T - K),
+           "ramp_nvfp4_arc": [arc.STEP_NVFP4] * K + [arc.STEP_BF16] * (T - K),
+           "uniform_fp8": [arc.STEP_FP8] * T}
+    res, ref = {}, None
+    for name, fmts in sch.items():
+        with torch.cuda.stream(stream):
+            h.copy_(h0)
+            arc.recurrent_prefill_schedule(h, blk, fmts, workspace=wsp, stream=stream)
+            out = h.float().clone()
+            ts = []
+            for _ in range(reps):
+                flush_l2(flush)
+                h.copy_(h0)
+                a, b = _ev(), _ev()
+                a.record(stream)
+                arc.recurrent_prefill_schedule(h, blk, fmts, workspace=wsp, stream=stream)
+                b.record(stream)
+                ts.append((a, b))
+        stream.synchronize()
+        if ref is None:
+            ref = out
+        res[name] = {"ms": statistics.median(a.elapsed_time(b) for a, b in ts),
+                     "hidden_state_rel_err_vs_all_bf16": (torch.linalg.norm(out - ref) / torch.linalg.norm(ref)).item()}
+    for name in res:
+        res[name]["speedup_vs_all_bf16"] = res["all_bf16"]["ms"] / res[name]["ms"]
+    if arc.last_device_status(stream) != 0:
+        raise RuntimeError("device status set during the RAMP instantiations")
+    return res
 
 
 def schedule_study(arc, h, h0, blk, wsp, flush, stream, T, budget, ref, device, reps=5):
@@ -779,6 +826,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
     ap.add_argument("--proj", default="all", help="profiling: run only this layer (e.g. qkv, gateup)")
+    ap.add_argument("--no-studies", action="store_true",
+                    help="recurrent workload: the k_low sweep only (no schedule, RAMP T=32 or contractive study)")
     ap.add_argument("--format", default="nvfp4", choices=["nvfp4", "mxfp4", "fp8"],
                     help="linear-layer workloads: NVFP4 + ARC (default), MXFP4 + ARC (32-value blocks, "
                          "power-of-two scales, no tensor scale) or FP8 W8A8 with per-tensor scales")

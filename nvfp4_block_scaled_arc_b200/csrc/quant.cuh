@@ -14,14 +14,13 @@
 //   k_amax        (dynamic scale, no RMSNorm) streams X once: max |x|, one partial per CTA
 //   k_row_stats   (RMSNorm prologue) one warp per row: exact sum of squares -> 1/rms (double);
 //                 with a dynamic scale also max |RMSNorm(x)|, one partial per CTA
-//   k_quant_rows  one CTA per row at a time, every thread two 16-element blocks in flight: block scale,
-//                 E2M1 codes, scale byte (four neighbouring lanes' bytes gathered into one
-//                 32-bit store in the swizzled layout); once the row's K channels are done, the
-//                 CTA forms the residual (activations) or value (weights) of each outlier
-//                 channel from the blocks holding outliers, which the coding threads kept in
-//                 shared memory (values, codes, d), stages them in its stash, codes the r/16
-//                 appended blocks and zero-fills the padding up to K_pad. A row never leaves its
-//                 CTA, so no grid-wide synchronisation is needed.
+//   k_quant_rows  one warp per row at a time, lane l coding blocks 32j + l (the row's next 32-block
+//                 segment loaded while one is coded): block scale, E2M1 codes, scale byte; once
+//                 the row's K channels are done, the warp forms the residual (activations) or
+//                 value (weights) of each outlier channel from the blocks holding outliers, whose
+//                 codes and d its lanes kept in shared memory, stages them in its stash, codes the
+//                 r/16 appended blocks and zero-fills the padding up to K_pad. A row never leaves
+//                 its warp, so no grid-wide synchronisation is needed.
 //   k_quant_reordered  the same coding with the channels in calibration order: rows staged in
 //                 shared memory by 1-D bulk copies, each block gathered through the permutation,
 //                 appended block j formed from primary block j in registers.
