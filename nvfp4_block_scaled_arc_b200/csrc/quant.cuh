@@ -451,6 +451,26 @@ __global__ void __launch_bounds__(kQRowMaxWarps * 32, 4) k_quant_rows(QuantArgs 
   uint4* slots = reinterpret_cast<uint4*>(wsm);
   float* stash = reinterpret_cast<float*>(wsm + static_cast<size_t>(nslot) * 16);
 
+  // Rows of this warp: m = blockIdx.x + gridDim.x * j for j = warp, warp + nwarps, ... The row's
+  // 32-block segments are double-buffered in registers: segment s + 1 (or the next row's first
+  // segment) is loaded while segment s is coded. The first segment is requested before anything
+  // else (X is not written by the first kernel), so its latency overlaps the set-up below.
+  const __nv_bfloat16* __restrict__ xg = a.x;
+  auto row_of = [&](int64_t jj) { return static_cast<int64_t>(blockIdx.x) + static_cast<int64_t>(gridDim.x) * jj; };
+  auto load_seg = [&](int64_t m, int seg, uint4& lo, uint4& hi) {
+    const int b = seg * 32 + lane;
+    lo = hi = make_uint4(0, 0, 0, 0);
+    if (m < a.M && b < nblk) {
+      const __nv_bfloat16* p = xg + m * a.ldx + 16 * b;
+      lo = ld_nc_v4_l1(p);
+      hi = ld_nc_v4_l1(p + 8);
+    }
+  };
+  int64_t jrow = warp;
+  int64_t m = row_of(jrow);
+  uint4 cur_lo, cur_hi;
+  load_seg(m, 0, cur_lo, cur_hi);
+
   // ---- outlier tables (before the wait: they overlap the first kernel); out-of-range entries
   // are reported and left out
   if (r > 0) {
@@ -500,24 +520,6 @@ __global__ void __launch_bounds__(kQRowMaxWarps * 32, 4) k_quant_rows(QuantArgs 
   const int nres = r >> 4, ntail = (a.kpad - a.K) >> 4;
   const bool keep_slots = r > 0 && !a.dup;  // activations need the codes and d of outlier blocks
 
-  // Rows of this warp: m = blockIdx.x + gridDim.x * j for j = warp, warp + nwarps, ... The row's
-  // 32-block segments are double-buffered in registers: segment s + 1 (or the next row's first
-  // segment) is loaded while segment s is coded.
-  const __nv_bfloat16* __restrict__ xg = a.x;
-  auto row_of = [&](int64_t jj) { return static_cast<int64_t>(blockIdx.x) + static_cast<int64_t>(gridDim.x) * jj; };
-  auto load_seg = [&](int64_t m, int seg, uint4& lo, uint4& hi) {
-    const int b = seg * 32 + lane;
-    lo = hi = make_uint4(0, 0, 0, 0);
-    if (m < a.M && b < nblk) {
-      const __nv_bfloat16* p = xg + m * a.ldx + 16 * b;
-      lo = ld_nc_v4_l1(p);
-      hi = ld_nc_v4_l1(p + 8);
-    }
-  };
-  int64_t jrow = warp;
-  int64_t m = row_of(jrow);
-  uint4 cur_lo, cur_hi;
-  load_seg(m, 0, cur_lo, cur_hi);
   for (; m < mpad; m = row_of(jrow += nwarps)) {
     // scale byte of (m, kb) at sf_row + (kb / 4) * 512 + kb % 4
     uint8_t* sf_row = a.sf + (m >> 7) * a.katoms * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4;
@@ -582,11 +584,11 @@ __global__ void __launch_bounds__(kQRowMaxWarps * 32, 4) k_quant_rows(QuantArgs 
       // ---- outlier channels: residual x - E2M1(code) * d (activations) or the value itself
       // (weights); with the prologue, x is normalised again exactly as the primary pass did
       __syncwarp();
-      auto residual = [&](int jj, int c, uint32_t hb) {
+      auto residual = [&](int jj, int c, uint32_t hb, uint32_t gbits) {
         float res = 0.0f;
         if (c >= 0) {
           float xv = __uint_as_float(hb << 16);
-          if (RMS) xv = rms_apply(xv, inv, __uint_as_float(ldg_nc_u16(a.gain + c) << 16));
+          if (RMS) xv = rms_apply(xv, inv, __uint_as_float(gbits << 16));
           res = xv;
           if (!a.dup) {
             const uint4 meta = slots[blk_slot[c >> 4]];
@@ -597,9 +599,21 @@ __global__ void __launch_bounds__(kQRowMaxWarps * 32, 4) k_quant_rows(QuantArgs 
         }
         stash[jj] = res;
       };
-      for (int jj = lane; jj < r; jj += 32) {
-        const int c = idx_s[jj];
-        residual(jj, c, c >= 0 ? ldg_nc_u16(row + c) : 0u);
+      // four iterations' channel loads are issued together, so their latencies overlap
+      for (int j0 = 0; j0 < r; j0 += 128) {
+        int c[4];
+        uint32_t hb[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) c[u] = (j0 + 32 * u + lane < r) ? idx_s[j0 + 32 * u + lane] : -1;
+        uint32_t gb[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          hb[u] = c[u] >= 0 ? ldg_nc_u16(row + c[u]) : 0u;
+          if (RMS && c[u] >= 0) gb[u] = ldg_nc_u16(a.gain + c[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (j0 + 32 * u + lane < r) residual(j0 + 32 * u + lane, c[u], hb[u], gb[u]);
       }
       __syncwarp();
     }
