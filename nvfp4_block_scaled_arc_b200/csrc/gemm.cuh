@@ -123,6 +123,7 @@ struct GemmArgs {
   int katoms;   // fp4: 512-byte scale atoms per 128-row block (K_pad / 64)
   int nblk128;  // fp4: 128-row blocks of B's scales (ceil(N / 128))
   int tiles_m, tiles_n;
+  int group_m;  // raster: consecutive tiles walk group_m row blocks before the next column block
   int box_rows_a, box_rows_b;  // TMA box heights (min(128, M), min(256, N))
   const uint8_t* sfa;
   const uint8_t* sfb;
@@ -136,8 +137,10 @@ struct GemmArgs {
   int inject;
 };
 
-__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int& tm, int& tn) {
-  constexpr int GM = 16;  // consecutive tiles walk 16 row blocks before moving to the next column block
+// Grouped raster: tiles t = 0, 1, ... walk GM row blocks of one column block, then the same row
+// blocks of the next column block, and so on; then the next group of row blocks. A group's A
+// rows stay in L2 while B streams through it once per group.
+__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int GM, int& tm, int& tn) {
   const int per_group = GM * tiles_n;
   const int group = t / per_group;
   const int first_m = group * GM;
@@ -217,7 +220,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         int tm, tn;
-        tile_coords(t, g.tiles_m, g.tiles_n, tm, tn);
+        tile_coords(t, g.tiles_m, g.tiles_n, g.group_m, tm, tn);
         for (int ks = 0; ks < g.kstages; ++ks) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, g.wait_ns, abort_flag)) {
             ok = false;
@@ -406,7 +409,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t acc = 0, acc_phase = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
       int tm, tn;
-      tile_coords(t, g.tiles_m, g.tiles_n, tm, tn);
+      tile_coords(t, g.tiles_m, g.tiles_n, g.group_m, tm, tn);
       const int row = tm * T::BM + q * 32 + lane;
       const bool row_ok = row < g.M;
       const int col0 = tn * T::BN + half * HB;

@@ -329,6 +329,15 @@ arc_status gemm_launch(const CUtensorMap& ta, const CUtensorMap& tb, GemmArgs g,
                        cudaStream_t s) {
   const int ntiles = g.tiles_m * g.tiles_n;
   const unsigned grid = static_cast<unsigned>(std::min(ntiles, sms));
+  // raster groups: as many 128-row blocks of A as fit in about 36 MB (well inside the 126 MB L2,
+  // beside the streaming B block and output), split into groups of equal size; B is then read
+  // from HBM once per group
+  {
+    const int64_t a_row_bytes = static_cast<int64_t>(g.ksteps) * (KIND == arc::kGemmFP4 ? 36 : KIND == arc::kGemmMX4 ? 34 : 32);
+    const int64_t gm_max = std::max<int64_t>(1, (36ll << 20) / (128 * a_row_bytes));
+    const int64_t ngroups = (g.tiles_m + gm_max - 1) / gm_max;
+    g.group_m = static_cast<int>((g.tiles_m + ngroups - 1) / ngroups);
+  }
   const int smem = arc::gemm_smem_bytes<KIND>();
   CUtensorMap ty;
   std::memset(&ty, 0, sizeof(ty));
