@@ -146,3 +146,65 @@ def test_rejects_bad_arguments():
     idx = torch.arange(17, dtype=torch.int32, device="cuda")
     with pytest.raises(arc.ArcError):
         arc.quantize_act_nvfp4(x, idx)  # r % 16 != 0
+
+
+def test_graph_capture_and_replay_give_identical_bytes():
+    # The quantizer captured in a CUDA graph (abs-max partials, then the coding kernel started by
+    # programmatic dependent launch) and replayed twice gives the bytes of a direct call, and
+    # both equal the oracle.
+    d = W.llama8b("qkv", rows=300, with_w=False)
+    x_bits = d["x"]
+    idx = O.calibrate(x_bits, 128)
+    x = to_dev(x_bits)
+    d_idx = torch.from_numpy(idx).cuda()
+    direct = arc.quantize_act_nvfp4(x, d_idx)
+    out = arc.quantize_act_nvfp4(x, d_idx)  # the buffers the graph writes
+    ws = torch.empty(arc.quantize_workspace_bytes(300, 128), dtype=torch.uint8, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        arc.quantize_act_nvfp4(x, d_idx, out=out, workspace=ws, stream=side)  # warm-up outside capture
+        torch.cuda.synchronize()
+        for t in (out.codes, out.sf, out.scale):
+            t.zero_()
+        with torch.cuda.graph(g, stream=side):
+            arc.quantize_act_nvfp4(x, d_idx, out=out, workspace=ws, stream=side)
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert arc.last_device_status() == 0
+    assert torch.equal(out.codes, direct.codes) and torch.equal(out.sf, direct.sf)
+    assert out.scale.item() == direct.scale.item()
+    s_ref = O.tensor_scale(O.amax(x_bits))
+    c_ref, sf_ref = O.quantize_act(x_bits, idx, s_ref)
+    assert_codes_equal(gpu_codes(out, 300), c_ref, "codes")
+    assert_codes_equal(gpu_sf_canonical(out, 300), sf_ref, "scale bytes")
+
+
+@pytest.mark.parametrize("rows,proj,static", [(1776, "down", None), (9473, "qkv", None), (9473, "qkv", 0.02)])
+def test_many_rows_per_warp(rows, proj, static):
+    # several rows per warp (each warp codes rows blockIdx + gridDim * j), with the next row's
+    # first segment prefetched across the row boundary, and a ragged row count past one full
+    # wave of rows
+    d = W.llama8b(proj, rows=rows, with_w=False)
+    run_and_compare(d["x"], r=128, static=static)
+
+
+def test_repeated_calls_with_one_workspace():
+    # consecutive calls reuse the workspace's abs-max partials: each call must see only its own
+    # maxima (a different tensor scale every call)
+    x0 = W.llama8b("o", rows=512, with_w=False)["x"]
+    idx = O.calibrate(x0, 64)
+    d_idx = torch.from_numpy(idx).cuda()
+    ws = torch.empty(arc.quantize_workspace_bytes(512, 64), dtype=torch.uint8, device="cuda")
+    for k, scale in enumerate((1.0, 4.0, 0.25, 8.0)):  # powers of two: exact in bf16
+        xb = (torch.from_numpy(O.bf16_bits_to_f32(x0)) * scale).bfloat16().view(torch.int16).numpy().view(np.uint16)
+        q = arc.quantize_act_nvfp4(to_dev(xb), d_idx, workspace=ws)
+        torch.cuda.synchronize()
+        assert arc.last_device_status() == 0
+        s_ref = O.tensor_scale(O.amax(xb))
+        assert q.scale.item() == np.float32(s_ref), (k, q.scale.item(), s_ref)
+        c_ref, sf_ref = O.quantize_act(xb, idx, s_ref)
+        assert_codes_equal(gpu_codes(q, 512), c_ref, "codes")
+        assert_codes_equal(gpu_sf_canonical(q, 512), sf_ref, "scale bytes")
