@@ -209,6 +209,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // everything above overlaps the previous kernel's tail; nothing below runs before it is done
+  pdl_wait();
   const uint32_t tmem = *tmem_slot;
   const int ntiles = g.tiles_m * g.tiles_n;
 

@@ -344,11 +344,21 @@ arc_status gemm_launch(const CUtensorMap& ta, const CUtensorMap& tb, GemmArgs g,
   if (!add && !make_store_map(&ty, g.y, static_cast<uint64_t>(g.N), static_cast<uint64_t>(g.M),
                               static_cast<uint64_t>(g.ldy) * 2))
     return ARC_ERR_CUDA;
-  if (add)
-    arc::k_gemm<KIND, true><<<grid, arc::kGemmThreads, smem, s>>>(ta, tb, ty, g);
-  else
-    arc::k_gemm<KIND, false><<<grid, arc::kGemmThreads, smem, s>>>(ta, tb, ty, g);
-  return launch_status();
+  // programmatic dependent launch: the set-up (tensor memory, barriers, descriptor prefetch)
+  // overlaps the tail of the kernel before it; the kernel waits for it before any other work
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(arc::kGemmThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = add ? cudaLaunchKernelEx(&cfg, arc::k_gemm<KIND, true>, ta, tb, ty, g)
+                            : cudaLaunchKernelEx(&cfg, arc::k_gemm<KIND, false>, ta, tb, ty, g);
+  return e == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
 }
 
 }  // namespace

@@ -299,8 +299,6 @@ __global__ void __launch_bounds__(256) k_row_stats(const __nv_bfloat16* __restri
 // ---------------------------------------------------------------------------------------------
 // Programmatic dependent launch: the quantizer's second kernel may start while the first one
 // runs; it waits here before it reads the first one's results.
-__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 constexpr int kAmaxSeg = 2048;  // elements of a row per warp work item
 
@@ -441,6 +439,7 @@ __device__ __forceinline__ void code_block_general(const float* v, float s, uint
 template <bool RMS>
 __global__ void __launch_bounds__(kQRowMaxWarps * 32, 4) k_quant_rows(QuantArgs a, int mpad) {
   extern __shared__ __align__(16) uint8_t qsm[];
+  pdl_launch_dependents();  // the GEMM that follows may set itself up meanwhile
   const int nwarps = static_cast<int>(blockDim.x >> 5);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nblk = a.K >> 4, r = a.r;
@@ -724,6 +723,7 @@ struct QuantMxArgs {
 
 __global__ void __launch_bounds__(kQMxMaxWarps * 32, 4) k_quant_mx_rows(QuantMxArgs a, int mpad) {
   extern __shared__ __align__(16) uint8_t qsm[];
+  pdl_launch_dependents();  // the GEMM that follows may set itself up meanwhile
   const int nwarps = static_cast<int>(blockDim.x >> 5);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nblk = a.K >> 5, r = a.r;
