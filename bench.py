@@ -33,9 +33,12 @@ Variants of the linear-layer workloads:
 
 Metric: NVFP4 ARC GEMM TFLOP/s = sum over the step of 2*M*N*(K+r) / step time, with the fused
 activation quantizer's GB/s (read X + write codes + scale bytes) beside it.
-Timing: CUDA events on the launching stream around every step and every kernel call; the L2 is
-flushed before every timed step, outside the events (a 256 MiB buffer written, then read back, so
-the lines it leaves in L2 are clean). Multi-GPU: one process
+Timing: CUDA events on the launching stream; two timed passes of --steps steps each, the L2
+flushed before every step, outside the events (a 256 MiB buffer written, then read back, so the
+lines it leaves in L2 are clean). The first pass has events around each step only and gives the
+step time (value, ms_per_step): events between the kernels would add gaps of their own and keep a
+kernel from starting while the one before it finishes. The second pass has events around every
+kernel call and gives the per-kernel times (roofline, per_projection). Multi-GPU: one process
 per GPU, each rank runs the same step on its own token batch (weak scaling, no data-path
 collective); time = max over ranks.
 
@@ -336,6 +339,10 @@ def run_layers(args, rank, world, device, layers, with_error=False):
     if arc.last_device_status(stream) != 0:
         raise RuntimeError("device status set during warm-up")
 
+    # two timed passes of K steps each, the L2 flushed before every step: the first with events
+    # around each step only (the step's time: events between the kernels would add their own
+    # gaps and keep a kernel from starting while the one before it finishes), the second with
+    # events around every kernel call (the per-kernel times of the roofline)
     step_ev, kern = [], []
     _barrier(world)
     torch.cuda.synchronize(device)
@@ -345,10 +352,13 @@ def run_layers(args, rank, world, device, layers, with_error=False):
                 flush_l2(flush)
                 s0, s1 = _ev(), _ev()
                 s0.record(stream)
-                rec = []
-                step(rec)
+                step(None)
                 s1.record(stream)
                 step_ev.append((s0, s1))
+            for _ in range(args.steps):
+                flush_l2(flush)
+                rec = []
+                step(rec)
                 kern.append(rec)
         torch.cuda.synchronize(device)
     _barrier(world)
@@ -406,7 +416,7 @@ def run_layers(args, rank, world, device, layers, with_error=False):
     # the GEMM
     per_layer_launches = 2 if mx else 3
     return dict(total_ms=total_ms, q_ms=q_ms, g_ms=g_ms, e2e_ms=e2e_ms, per_layer=per_layer, clocks=clocks,
-                h2d=h2d, d2h=d2h, launches=args.steps * len(layers) * per_layer_launches)
+                h2d=h2d, d2h=d2h, launches=2 * args.steps * len(layers) * per_layer_launches)
 
 
 def layers_line(args, world, layers, desc, res):
@@ -429,6 +439,8 @@ def layers_line(args, world, layers, desc, res):
         "dtype": "e4m3 x e4m3 -> f32 (bf16 out)" if fp8 else "e2m1 x e2m1 -> f32 (bf16 out)",
         "data": "synthetic (seeded; random weights and activations of the stated shapes)",
         "config": {"workload": desc, "l2": "flushed before every step (256 MiB written, then read back)",
+                   "timing": "step time from a pass with events around each step only; kernel times from a "
+                             "second pass with events around every kernel call",
                    "parallelism": f"replicas x{world}",
                    "channel_order": "reordered by calibration abs-max" if getattr(args, "reorder", False)
                    else "natural (outlier list)"},

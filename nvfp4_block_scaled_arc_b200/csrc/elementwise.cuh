@@ -10,6 +10,7 @@ namespace arc {
 __global__ void __launch_bounds__(256) k_rmsnorm(const __nv_bfloat16* __restrict__ h, int64_t ldh, int M, int K,
                                                  const __nv_bfloat16* __restrict__ gain, double eps,
                                                  __nv_bfloat16* __restrict__ out, int64_t ldo) {
+  pdl_launch_dependents();  // the GEMM that follows may set itself up meanwhile
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m = blockIdx.x * 8 + warp;
   if (m >= M) return;
@@ -34,6 +35,7 @@ __global__ void __launch_bounds__(256) k_rmsnorm(const __nv_bfloat16* __restrict
 // in fp32 (expf, IEEE divide and multiply). 8 columns per thread, F % 8 == 0.
 __global__ void __launch_bounds__(256) k_silu_mul(const __nv_bfloat16* __restrict__ gu, int64_t ld, int M, int F,
                                                   __nv_bfloat16* __restrict__ out, int64_t ldo) {
+  pdl_launch_dependents();  // the GEMM that follows may set itself up meanwhile
   const int vpr = F >> 3;
   const int64_t total = static_cast<int64_t>(M) * vpr;
   for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < total;

@@ -877,6 +877,7 @@ template <bool RMS>
 __global__ void __launch_bounds__(kQReoThreads, 3) k_quant_reordered(QuantArgs a, const int32_t* __restrict__ perm,
                                                                      int mpad) {
   extern __shared__ __align__(128) uint8_t qreo_smem[];
+  pdl_launch_dependents();  // the GEMM that follows may set itself up meanwhile
   constexpr int NT = kQReoThreads;
   const int nblk = a.K >> 4;
   const int tid = threadIdx.x, lane = tid & 31;
@@ -1086,6 +1087,7 @@ __device__ __forceinline__ uint32_t e4m3x2_rn_sat(float lo, float hi) {
 __global__ void __launch_bounds__(256) k_quant_fp8(const __nv_bfloat16* __restrict__ x, int64_t ldx, int M, int K,
                                                    const float* static_scale, const uint32_t* partials,
                                                    int npartials, float* scale_out, uint8_t* codes, int64_t ldc) {
+  pdl_launch_dependents();  // the GEMM that follows may set itself up meanwhile
   pdl_wait();
   float s;
   {
