@@ -386,17 +386,37 @@ def run_layers(args, rank, world, device, layers, with_error=False):
         h2d = sum(v.numel() * 2 for v in xs_pin.values())
         d2h = sum(v.numel() * 2 for v in ys_pin.values())
 
-        def e2e_step():
+        # three streams: host-to-device copies, compute, device-to-host copies. Within a step the
+        # upload of the next projection's X and the download of the previous Y overlap the
+        # compute (PCIe is full duplex); events order each copy against the work that uses it.
+        # A step starts after its start event and ends after its last download.
+        up, down = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
+        x_ready = {L["name"]: torch.cuda.Event() for L in layers}
+        y_ready = {L["name"]: torch.cuda.Event() for L in layers}
+
+        def e2e_step(start):
+            up.wait_event(start)
             for L in layers:
                 name = L["name"]
-                xs[name].copy_(xs_pin[name], non_blocking=True)
+                with torch.cuda.stream(up):
+                    xs[name].copy_(xs_pin[name], non_blocking=True)
+                x_ready[name].record(up)
+            for L in layers:
+                name = L["name"]
+                stream.wait_event(x_ready[name])
                 quant(name, out=qa[name], workspace=wsp[name])
                 gemm(qa[name], packed[name], out=ys[name], stream=stream)
-                ys_pin[name].copy_(ys[name], non_blocking=True)
+                y_ready[name].record(stream)
+                down.wait_event(y_ready[name])
+                with torch.cuda.stream(down):
+                    ys_pin[name].copy_(ys[name], non_blocking=True)
+            stream.wait_stream(down)
 
         with torch.cuda.stream(stream):
             for _ in range(max(1, min(args.warmup, 2))):
-                e2e_step()
+                s0 = _ev()
+                s0.record(stream)
+                e2e_step(s0)
         stream.synchronize()
         _barrier(world)
         e2e_ev = []
@@ -404,7 +424,7 @@ def run_layers(args, rank, world, device, layers, with_error=False):
             for _ in range(args.steps):
                 a, b = _ev(), _ev()
                 a.record(stream)
-                e2e_step()
+                e2e_step(a)
                 b.record(stream)
                 e2e_ev.append((a, b))
         stream.synchronize()
