@@ -12,17 +12,19 @@
 //
 // CTA = 15 warps, one CTA per SM, persistent over 128 x 256 output tiles (grouped raster):
 //   warp 0       TMA producer: per stage an A tile of 128 rows x 128 bytes and a B tile of 256
-//                rows x 128 bytes (128-byte swizzle), plus the stage's scale atoms as 1-D bulk
-//                copies (A: up to 4 atoms of its 128-row block; B: up to 4 atoms of each of its
-//                two 128-row blocks); no multicast.
+//                rows x 128 bytes (128-byte swizzle), plus A's scale atoms of the stage as a 1-D
+//                bulk copy (up to 4 atoms of its 128-row block); it arms the stage's barrier with
+//                all of the stage's bytes, B's scale atoms (warp 2) included; no multicast.
 //   warp 1       MMA issue, one thread, every pipeline stage in order: the fp32 accumulation
 //                order is fixed, so results are reproducible bit for bit. The issuing thread
 //                does no release/acquire memory operation: one such pair per stage in this
 //                thread costs about 40% of the tensor pipe's throughput (measured with the MMA
 //                issue loop alone, 7.1 against 5.1 PFLOP/s), while tcgen05 fences cost nothing.
 //                Warp 1 also owns the TMEM allocation.
-//   warp 2       idle (keeps the scale writers and epilogue warps on the TMEM lane quarters
-//                their warp index selects).
+//   warp 2       (FP4) issues each stage's bulk copies of B's scale atoms, beside the producer's
+//                operand and A-scale copies: two small copies fewer in the producer's sequence
+//                make the stages land sooner (7 % on gateup). Its position also keeps the scale
+//                writers and epilogue warps on the TMEM lane quarters their warp index selects.
 //   warps 3..6   (FP4) scale writers, one per TMEM lane quarter: they read the stage's scale
 //                bytes from shared memory and store them into the stage's set of TMEM scale
 //                columns with tcgen05.st, in the cell order the block-scaled MMA reads
@@ -249,9 +251,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               uint8_t* sSFA = sB + T::B_BYTES;
               uint8_t* sSFB = sSFA + T::SFA_BYTES;
               bulk_load(sSFA, g.sfa + (static_cast<int64_t>(tm) * g.katoms + APS * ks) * 512, natoms * 512, &full[stage]);
-              for (int b = 0; b < nb; ++b)
-                bulk_load(sSFB + b * APS * 512, g.sfb + (static_cast<int64_t>(2 * tn + b) * g.katoms + APS * ks) * 512,
-                          natoms * 512, &full[stage]);
+              (void)sSFB;  // B's scale atoms: warp 2
             }
             armed |= 1u << stage;
             armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
@@ -321,7 +321,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_wait_teardown(drain, 0, g.wait_ns);
     }
   } else if (warp == 2) {
-    // idle
+    if (FP4 && lane == 0) {
+      // B's scale atoms of every stage, issued beside the producer's copies
+      constexpr int APS = MX4 ? 2 : 4;
+      uint32_t stage = 0, phase = 0, armed = 0, armed_par = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        int tm, tn;
+        tile_coords(t, g.tiles_m, g.tiles_n, g.group_m, tm, tn);
+        (void)tm;
+        for (int ks = 0; ks < g.kstages; ++ks) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, g.wait_ns, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int natoms = min(APS, g.katoms - APS * ks);
+          const int nb = min(2, g.nblk128 - 2 * tn);
+          uint8_t* sSFB = smem + stage * T::STAGE_BYTES + T::A_BYTES + T::B_BYTES + T::SFA_BYTES;
+          for (int b = 0; b < nb; ++b)
+            bulk_load(sSFB + b * APS * 512, g.sfb + (static_cast<int64_t>(2 * tn + b) * g.katoms + APS * ks) * 512,
+                      natoms * 512, &full[stage]);
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == T::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (*abort_flag) {
+        for (int s = 0; s < T::STAGES; ++s)
+          if ((armed >> s) & 1u) mbar_wait_teardown(&full[s], (armed_par >> s) & 1u, g.wait_ns);
+      }
+    }
   } else if (warp < kGemmEpiWarp0) {
     if (FP4) {
       // ------------------------------------------------------------------ scale writers
