@@ -164,6 +164,23 @@ __device__ __forceinline__ uint4 lds_u32x4(uint32_t addr) {
   return v;
 }
 
+// One MMA of a pipeline stage: K-step k of the stage, operand descriptors already offset to it
+// (32 bytes of K per step = 2 descriptor units), scales (block-scaled kinds) from the stage's set:
+// A's at sf + 32 + 4k, B's at sf + 8k.
+template <int KIND>
+__device__ __forceinline__ void mma_step(uint32_t d_tmem, uint64_t da, uint64_t db, uint32_t sf, int k,
+                                         uint32_t accum) {
+  using T = GemmTraits<KIND>;
+  if constexpr (KIND == kGemmFP4)
+    tc_mma_nvf4(d_tmem, da, db, T::IDESC, sf + 32 + 4 * k, sf + 8 * k, accum);
+  else if constexpr (KIND == kGemmMX4)
+    tc_mma_mxf4(d_tmem, da, db, T::IDESC, sf + 32 + 4 * k, sf + 8 * k, accum);
+  else if constexpr (KIND == kGemmFP8)
+    tc_mma_f8(d_tmem, da, db, T::IDESC, accum);
+  else
+    tc_mma_bf16(d_tmem, da, db, T::IDESC, accum);
+}
+
 constexpr int kGemmThreads = 480;  // producer, MMA issuer, idle warp, 4 scale writers, 8 epilogue warps
 constexpr int kGemmEpiWarp0 = 7;
 
@@ -271,9 +288,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------------ MMA issue
+      // Each tcgen05.mma is accepted only about as fast as the tensor pipe runs them, so every
+      // instruction between two MMAs lengthens the pipe's idle time at a stage boundary: the
+      // stage's descriptors and scale columns are advanced by one add each, and the four MMAs of
+      // a full stage are unrolled (5 % on the llama8b projections against recomputing them).
       uint32_t acc = 0, acc_phase = 0;
       uint32_t stage = 0, phase = 0;  // the same stage sequence the producer walks
       bool ok = true;
+      constexpr uint64_t kStageDesc = static_cast<uint64_t>(T::STAGE_BYTES >> 4);  // descriptor units
+      constexpr uint64_t kBDesc = static_cast<uint64_t>(T::A_BYTES >> 4);
+      const uint64_t da0 = desc_kmajor_sw128(smem_u32(smem));
+      uint64_t da = da0;                 // stage's A tile; its B tile at da + kBDesc
+      uint32_t sf = tmem + T::SF_COL0;   // stage's scale set
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         // the accumulator must have been drained by the epilogue
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, g.wait_ns, abort_flag)) break;
@@ -285,28 +311,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           tc_fence_after();
-          uint8_t* sA = smem + stage * T::STAGE_BYTES;
-          uint8_t* sB = sA + T::A_BYTES;
-          const int nk = (FP4 || FP8) ? min(4, g.ksteps - 4 * ks) : 4;  // MMAs in this stage
-          const uint64_t da = desc_kmajor_sw128(smem_u32(sA));
-          const uint64_t db = desc_kmajor_sw128(smem_u32(sB));
-          const uint32_t sf = tmem + T::SF_COL0 + T::SF_SET_COLS * stage;
-          for (int k = 0; k < nk; ++k) {
-            const uint64_t off = static_cast<uint64_t>((k * 32) >> 4);
-            const uint32_t accum = (ks > 0 || k > 0) ? 1u : 0u;
-            if (NV4)
-              tc_mma_nvf4(d_tmem, da + off, db + off, T::IDESC, sf + 32 + 4 * k, sf + 8 * k, accum);
-            else if (MX4)
-              tc_mma_mxf4(d_tmem, da + off, db + off, T::IDESC, sf + 32 + 4 * k, sf + 8 * k, accum);
-            else if (FP8)
-              tc_mma_f8(d_tmem, da + off, db + off, T::IDESC, accum);
-            else
-              tc_mma_bf16(d_tmem, da + off, db + off, T::IDESC, accum);
+          const uint64_t db = da + kBDesc;
+          const uint32_t acc0 = ks > 0 ? 1u : 0u;  // the tile's first MMA overwrites
+          // MMAs in this stage: 4 of K = 64 (FP4) / K = 32 (FP8) / K = 16 (BF16), fewer at the end
+          const int nk = (FP4 || FP8) ? min(4, g.ksteps - 4 * ks) : 4;
+          if (nk == 4) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mma_step<KIND>(d_tmem, da + 2 * k, db + 2 * k, sf, k, k > 0 ? 1u : acc0);
+          } else {
+            for (int k = 0; k < nk; ++k) mma_step<KIND>(d_tmem, da + 2 * k, db + 2 * k, sf, k, k > 0 ? 1u : acc0);
           }
           tc_commit(&empty[stage]);
           if (++stage == T::STAGES) {
             stage = 0;
             phase ^= 1u;
+            da = da0;
+            sf = tmem + T::SF_COL0;
+          } else {
+            da += kStageDesc;
+            sf += T::SF_SET_COLS;
           }
         }
         if (!ok) break;
