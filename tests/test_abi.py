@@ -113,3 +113,28 @@ def test_static_scratch_reports_argument_errors_before_its_size_limit(L):
                                                    fake, None) == 2  # misaligned codes
     assert L.arc_quantize_act_nvfp4_static_scratch(fake, big, 64, 64, None, 0, None, 1e-6, None, fake, fake, fake,
                                                    None) == 6  # well-formed, too large
+
+
+def test_host_checks_of_the_mxfp4_calls(L):
+    P = ctypes.c_void_p
+    fake, idx = P(0x10000), P(0x30000)
+    q, w = L.arc_quantize_act_mxfp4, L.arc_pack_weight_mxfp4
+    for f in (q, w):
+        # K % 32 != 0, r % 32 != 0, r > K, NULL idx with r > 0, NULL output, ld < K
+        assert f(fake, 4, 48, 48, None, 0, fake, fake, None) == 1
+        assert f(fake, 4, 64, 64, idx, 16, fake, fake, None) == 1
+        assert f(fake, 4, 64, 64, idx, 96, fake, fake, None) == 1
+        assert f(fake, 4, 64, 64, None, 32, fake, fake, None) == 1
+        assert f(fake, 4, 64, 64, None, 0, None, fake, None) == 1
+        assert f(fake, 4, 64, 32, None, 0, fake, fake, None) == 1
+        # misaligned input rows or outputs
+        assert f(P(0x10008), 4, 64, 64, None, 0, fake, fake, None) == 2
+        assert f(fake, 4, 64, 68, None, 0, fake, fake, None) == 2
+        assert f(fake, 4, 64, 64, None, 0, fake, P(0x10004), None) == 2
+    g = L.arc_gemm_mxfp4
+    # N % 8 != 0, ldy < N, ld_add < N with an add term, NULL operand, misaligned output
+    assert g(fake, fake, fake, fake, 4, 12, 64, fake, 16, None, 0, None) == 1
+    assert g(fake, fake, fake, fake, 4, 16, 64, fake, 8, None, 0, None) == 1
+    assert g(fake, fake, fake, fake, 4, 16, 64, fake, 16, fake, 8, None) == 1
+    assert g(None, fake, fake, fake, 4, 16, 64, fake, 16, None, 0, None) == 1
+    assert g(fake, fake, fake, fake, 4, 16, 64, P(0x10002), 16, None, 0, None) == 2
