@@ -140,7 +140,9 @@ arc_status arc_pack_weight_nvfp4(const void* w_bf16, int64_t N, int64_t K, int64
 /*
  * Offline outlier identification ("Adaptieve Uitschieter-identificatie"): the r channels of the
  * calibration tensor X [M, K] with the largest abs-max, in descending order, ties by ascending
- * index, written to d_idx_out (device int32[r]). 0 < r <= K, r <= 1024.
+ * index, written to d_idx_out (device int32[r]). 0 < r <= K, r <= 1024, K even, ldx even and x
+ * 4-byte aligned (else ARC_ERR_INVALID_ARG / ARC_ERR_ALIGNMENT); workspace of at least
+ * arc_calibrate_workspace_bytes(K), 256-byte aligned (else ARC_ERR_WORKSPACE / ARC_ERR_ALIGNMENT).
  */
 arc_status arc_calibrate_outliers(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, int32_t r,
                                   int32_t* d_idx_out, void* workspace, size_t ws_bytes, arc_stream_t stream);

@@ -138,3 +138,55 @@ def test_host_checks_of_the_mxfp4_calls(L):
     assert g(fake, fake, fake, fake, 4, 16, 64, fake, 16, fake, 8, None) == 1
     assert g(None, fake, fake, fake, 4, 16, 64, fake, 16, None, 0, None) == 1
     assert g(fake, fake, fake, fake, 4, 16, 64, P(0x10002), 16, None, 0, None) == 2
+
+
+def test_host_checks_of_calibration_and_the_elementwise_calls(L):
+    P = ctypes.c_void_p
+    fake, ws = P(0x10000), P(0x20000)
+    big = 1 << 20
+    c = L.arc_calibrate_outliers
+    assert c(fake, 4, 63, 64, 8, fake, ws, big, None) == 1      # K odd
+    assert c(fake, 4, 64, 64, 0, fake, ws, big, None) == 1      # r <= 0
+    assert c(fake, 4, 64, 64, 65, fake, ws, big, None) == 1     # r > K
+    assert c(fake, 4, 4096, 4096, 1025, fake, ws, big, None) == 1  # r > 1024
+    assert c(fake, 4, 64, 32, 8, fake, ws, big, None) == 1      # ldx < K
+    assert c(None, 4, 64, 64, 8, fake, ws, big, None) == 1
+    assert c(fake, 4, 64, 64, 8, None, ws, big, None) == 1
+    assert c(P(0x10002), 4, 64, 64, 8, fake, ws, big, None) == 2  # x not 4-byte aligned
+    assert c(fake, 4, 64, 64, 8, fake, ws, 8, None) == 6        # workspace too small
+    assert c(fake, 4, 64, 64, 8, fake, P(0x20010), big, None) == 2  # workspace not 256-byte aligned
+    n = L.arc_rmsnorm_bf16
+    assert n(fake, 4, 60, 64, fake, 1e-6, fake, 64, None) == 1   # d % 8
+    assert n(fake, 4, 64, 56, fake, 1e-6, fake, 64, None) == 1   # ldh < d
+    assert n(fake, 4, 64, 64, None, 1e-6, fake, 64, None) == 1   # no gain
+    assert n(fake, 4, 64, 64, fake, 1e-6, P(0x10008), 64, None) == 2
+    s = L.arc_silu_mul_bf16
+    assert s(fake, 4, 60, 128, fake, 64, None) == 1              # F % 8
+    assert s(fake, 4, 64, 120, fake, 64, None) == 1              # ld_gu < 2F
+    assert s(fake, 4, 64, 128, fake, 56, None) == 1              # ldo < F
+    assert s(P(0x10008), 4, 64, 128, fake, 64, None) == 2
+
+
+def test_size_queries_of_mxfp4_calibration_and_the_recurrence(L):
+    for rows, kaug in [(16, 272), (4096, 4224), (130, 14464), (1, 64), (129, 96), (300, 160)]:
+        # one UE8M0 scale per 32 values of the padded depth, in the same 512-byte atoms
+        assert L.arc_mxfp4_sf_bytes(rows, kaug) == O.sf_swizzled_bytes(rows, O.kpad(kaug) // 32)
+    assert L.arc_mxfp4_sf_bytes(0, 64) == 0 and L.arc_mxfp4_sf_bytes(4, 0) == 0
+    for K in (2, 256, 4096, 14336, 1000):
+        w = L.arc_calibrate_workspace_bytes(K)
+        assert w >= 12 * K and w % 256 == 0  # u32 column maxima + u64 sort keys
+    assert L.arc_calibrate_workspace_bytes(0) == 0
+    # the recurrence's workspace holds its codes, scale bytes, gate|up, activation, normed input
+    # and a quantizer workspace, each rounded up to 256 bytes
+    S, d, F, rg, rd = 4096, 2048, 8192, 64, 64
+    subs = (arc.SwigluSublayer * 2)()
+    for sl in subs:
+        sl.r_gateup, sl.r_down = rg, rd
+    blk = arc.SwigluBlock(d=d, ffn=F, eps=1e-6, n_sublayers=2, sublayers=subs)
+    w = L.arc_recurrent_workspace_bytes(S, ctypes.byref(blk))
+    parts = [max(L.arc_nvfp4_codes_bytes(S, d + rg), L.arc_nvfp4_codes_bytes(S, F + rd), S * max(d, F)),
+             max(L.arc_nvfp4_sf_bytes(S, d + rg), L.arc_nvfp4_sf_bytes(S, F + rd)), 8, S * 2 * F * 2, S * F * 2,
+             S * d * 2, L.arc_quantize_workspace_bytes(S, max(rg, rd))]
+    assert sum(parts) <= w <= sum(parts) + 7 * 256
+    assert L.arc_recurrent_workspace_bytes(0, ctypes.byref(blk)) == 0
+    assert L.arc_recurrent_workspace_bytes(S, None) == 0
